@@ -1,0 +1,477 @@
+"""Benchmark of the paged KV-cache attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl npv|reference] [--workload NAME]
+
+One step = one decode step of the workload: npv_store_kvcache of this step's
+new K/V rows, then npv_paged_decode_attention (split-KV kernel + merge kernel)
+over every sequence.  The default workload is the Qwen3-0.6B-shaped decode
+batch (256 sequences, 16 Q / 8 KV heads, head_dim 128, 256-token blocks,
+contexts U[100, 2048] growing by one token per step, cycling through its 64
+steps).  Inputs are synthetic and seeded; the KV read per step (about 1.16 GB)
+is far larger than the 126 MB L2, so no explicit flush is needed.
+
+`value` is algorithmic HBM bytes per step / device time per step (GB/s), summed
+over ranks for N > 1 (each rank runs its own replica; no collective on the data
+path) and divided by the slowest rank's time.  Prints one JSON line on rank 0.
+
+--impl reference times the fp64 CPU oracle (the only reference this method
+has) on a bounded sample of the same workload, on rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged GQA decode attention: achieved HBM GB/s (% of peak), tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+KERNEL_SRC = os.path.join(ROOT, "paged_kv_cache_bf16_b200", "csrc", "decode_attention.cuh")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["npv", "reference"], default="npv")
+    ap.add_argument("--workload", default="qwen3_decode")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline budget")
+    ap.add_argument("--ref-seconds", type=float, default=150.0, help="reference-arm budget")
+    return ap.parse_args(argv)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    with open(KERNEL_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the split kernel from the committed ncu summary,
+    or None if there is none or the kernel source changed since the capture."""
+    path = os.path.join(PROFILE_DIR, f"decode_split_{workload}.txt")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch_full_workload"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------------
+# workload bookkeeping (host side)
+# ---------------------------------------------------------------------------
+
+def step_bytes(wl, step):
+    """Algorithmic HBM bytes of one step: (store, decode attention)."""
+    row = wl.Hkv * wl.D * 2
+    T = wl.total_q
+    store = 2 * T * row * 2  # read key+value rows, write them into the caches
+    L = wl.context_lens(step).astype(np.int64)
+    qo = 2 * wl.total_q * wl.Hq * wl.D * 2  # read q, write out
+    meta = wl.B * 4 + int(sum(-(-int(x) // wl.BS) for x in L)) * 4
+    decode = int(L.sum()) * 2 * row + qo + meta
+    return store, decode
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling while the GPU is under load."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.t0 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.05)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for i, n in enumerate(names):
+                if r[5 + i].strip().lower() == "active":
+                    reasons.add(n)
+        # samples under load: the upper half of the observed clocks
+        loaded = sorted(sm)[len(sm) // 2:] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+
+class OracleRunner:
+    """Times the fp64 oracle on this workload's sequences, a sample at a time."""
+
+    def __init__(self, wl):
+        from oracle import oracle as O
+
+        self.O = O
+        self.wl = wl
+        self.threads = O.default_threads()
+        # compact pool: every block any step references, relabelled in order
+        last = wl.spec.num_steps - 1
+        bt = wl.block_tables(last)
+        used = np.unique(bt[bt >= 0])
+        self.lut = np.full(wl.NB, -1, dtype=np.int64)
+        self.lut[used] = np.arange(len(used))
+        shape = (len(used), wl.BS, wl.Hkv, wl.D)
+        self.kp = np.full(shape, 0x7FC0, dtype=np.uint16)
+        self.vp = np.full(shape, 0x7FC0, dtype=np.uint16)
+        ids, K, V = wl.prior_blocks_dense()
+        self.kp[self.lut[ids]] = K
+        self.vp[self.lut[ids]] = V
+        self.step_cache = {}
+
+    def inputs(self, step):
+        if step not in self.step_cache:
+            wl = self.wl
+            k, v = wl.new_kv(step)
+            slots = wl.slot_mapping(step).astype(np.int64)
+            cslots = (self.lut[slots // wl.BS] * wl.BS + slots % wl.BS).astype(np.int32)
+            bt = wl.block_tables(step)
+            btc = np.where(bt >= 0, self.lut[np.maximum(bt, 0)], -1).astype(np.int32)
+            self.step_cache[step] = (k, v, cslots, btc, wl.context_lens(step), wl.q(step))
+        return self.step_cache[step]
+
+    def run(self, step, seqs):
+        """Oracle store of every sequence's new token (so later steps read a
+        complete cache), then attention for the sampled sequences.  Returns the
+        algorithmic bytes of that work."""
+        wl = self.wl
+        k, v, cslots, btc, L, q = self.inputs(step)
+        seqs = np.asarray(seqs)
+        self.O.store_kvcache(k, v, self.kp, self.vp, cslots)
+        self.O.decode_attention(q[seqs], self.kp, self.vp, btc[seqs], L[seqs], threads=self.threads)
+        row = wl.Hkv * wl.D * 2
+        return (wl.B * 4 * row + len(seqs) * 2 * wl.Hq * wl.D * 2 +
+                int(L[seqs].astype(np.int64).sum()) * 2 * row)
+
+
+def cpu_baseline(wl, seconds: float):
+    runner = OracleRunner(wl)
+    # all sequences of successive steps, until the budget is spent
+    t0 = time.perf_counter()
+    nbytes = 0
+    steps = 0
+    while True:
+        nbytes += runner.run(steps % wl.spec.num_steps, np.arange(wl.B))
+        steps += 1
+        if time.perf_counter() - t0 >= seconds or steps >= wl.spec.num_steps:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": runner.threads, "kind": "oracle",
+            "tokens_per_s": steps * wl.B / dt,
+            "sample": f"fp64 C oracle (store + decode attention) on steps 0..{steps - 1} of {wl.spec.name}, "
+                      f"all {wl.B} sequences, {runner.threads} threads, {dt:.1f} s"}
+
+
+def reference_arm(args, rank, world):
+    from paged_kv_cache_bf16_b200 import workloads as W
+
+    if rank != 0:
+        return 0
+    wl = W.workload(args.workload)
+    runner = OracleRunner(wl)
+    # calibrate: seconds per sequence of oracle work
+    t0 = time.perf_counter()
+    runner.run(0, np.arange(min(8, wl.B)))
+    per_seq = (time.perf_counter() - t0) / min(8, wl.B)
+    total_steps = args.steps + args.warmup
+    n = int(max(1, min(wl.B, args.ref_seconds / max(1e-9, per_seq * total_steps))))
+    for i in range(args.warmup):
+        runner.run(i % wl.spec.num_steps, np.arange(i * n, i * n + n) % wl.B)
+    t0 = time.perf_counter()
+    nbytes = 0
+    for i in range(args.steps):
+        j = args.warmup + i
+        nbytes += runner.run(j % wl.spec.num_steps, (np.arange(n) + j * n) % wl.B)
+    dt = time.perf_counter() - t0
+    value = nbytes / dt / 1e9
+    sample = (f"each step: the fp64 C oracle's store + decode attention for {n} of the {wl.B} sequences of "
+              f"{wl.spec.name} ({runner.threads} threads)")
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(wl),
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": runner.threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(wl):
+    s = wl.spec
+    return {"workload": s.name, "num_seqs": s.num_seqs, "num_q_heads": s.num_q_heads,
+            "num_kv_heads": s.num_kv_heads, "head_dim": s.head_dim, "block_size": s.block_size,
+            "num_blocks": s.num_blocks, "context_lens": f"U[{s.ctx_lo},{s.ctx_hi}] +1 per step",
+            "steps_cycle": s.num_steps,
+            "l2": "not flushed: inputs larger than L2 (KV read per step ~1.2 GB vs 126 MB L2)"}
+
+
+# ---------------------------------------------------------------------------
+# the npv arm
+# ---------------------------------------------------------------------------
+
+def npv_arm(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from paged_kv_cache_bf16_b200 import ops
+    from paged_kv_cache_bf16_b200 import workloads as W
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    ops.lib()
+    wl = W.workload(args.workload)
+    nsteps = wl.spec.num_steps
+    st = W.DeviceState(wl, dev, steps=list(range(nsteps)))
+    ws = ops.alloc_workspace(ops.decode_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.D), dev)
+    out = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def store(i):
+        s = st.steps[i % nsteps]
+        ops.store_kvcache(s["key"], s["value"], st.k_cache, st.v_cache, s["slot_mapping"])
+
+    def decode(i):
+        s = st.steps[i % nsteps]
+        ops.paged_decode_attention(s["q"], st.k_cache, st.v_cache, s["block_tables"], s["context_lens"], out=out,
+                                   workspace=ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    bytes_steps = [step_bytes(wl, i % nsteps) for i in range(args.steps)]
+    store_bytes = sum(b[0] for b in bytes_steps)
+    decode_bytes = sum(b[1] for b in bytes_steps)
+
+    for i in range(args.warmup):
+        store(i)
+        decode(i)
+    ops.check_device_errors()
+
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+
+    # ---- timed region 1: the plain step loop -> value
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        store(i)
+        decode(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1))
+
+    # ---- timed region 2: the same loop with events around each decode call -> kernel roofline
+    barrier()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        store(i)
+        evs[i][0].record(stream)
+        decode(i)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    dec_ms = [a.elapsed_time(b) for a, b in evs]
+    dec_mean = max_over_ranks(sum(dec_ms) / len(dec_ms))
+
+    # keep the GPU loaded long enough for the clock sampler to see it
+    t_end = time.time() + 1.5
+    i = 0
+    while time.time() < t_end:
+        for _ in range(50):
+            store(i)
+            decode(i)
+            i += 1
+        torch.cuda.synchronize(dev)
+    clocks = sampler.stop() if sampler else None
+    ops.check_device_errors()
+
+    # ---- end to end through the public API, host buffers, copies timed
+    e2e = None
+    if not args.no_e2e:
+        e2e = npv_e2e(args, wl, st, ws, dev, stream, ops, W, barrier, max_over_ranks)
+
+    peak, peak_kind = measured_peaks()
+    total_bytes = (store_bytes + decode_bytes) * world
+    value = total_bytes / (ms * 1e-3) / 1e9
+    achieved = (decode_bytes / args.steps) / (dec_mean * 1e-3) / 1e9
+    traffic = profiled_traffic(args.workload)
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(wl),
+        "tokens_per_s": world * args.steps * wl.B / (ms * 1e-3),
+        "pct_of_peak_hbm": 100.0 * value / world / peak,
+        "roofline": {"kernel": "npv_paged_decode_attention (split-KV kernel + merge kernel)", "bound": "hbm",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                     else "fallback 6650 GB/s", "traffic": traffic,
+                     "algorithmic_bytes_per_launch": decode_bytes / args.steps,
+                     "mean_launch_ms": dec_mean},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def npv_e2e(args, wl, st, ws, dev, stream, ops, W, barrier, max_over_ranks):
+    """Host-resident inputs: each step copies its inputs H2D from pinned memory,
+    runs store + decode through the public API, and copies the output D2H."""
+    import torch
+
+    nsteps = wl.spec.num_steps
+    keys = ["q", "key", "value", "slot_mapping", "block_tables", "context_lens"]
+    host = []
+    for i in range(nsteps):
+        s = st.steps[i]
+        host.append({k: s[k].cpu().pin_memory() for k in keys})
+    dbuf = {k: torch.empty_like(st.steps[0][k]) for k in keys}
+    out_dev = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device=dev)
+    out_host = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16).pin_memory()
+    h2d = sum(host[0][k].numel() * host[0][k].element_size() for k in keys)
+    d2h = out_host.numel() * out_host.element_size()
+
+    def step(i):
+        h = host[i % nsteps]
+        for k in keys:
+            dbuf[k].copy_(h[k], non_blocking=True)
+        ops.store_kvcache(dbuf["key"], dbuf["value"], st.k_cache, st.v_cache, dbuf["slot_mapping"])
+        ops.paged_decode_attention(dbuf["q"], st.k_cache, st.v_cache, dbuf["block_tables"], dbuf["context_lens"],
+                                   out=out_dev, workspace=ws)
+        out_host.copy_(out_dev, non_blocking=True)
+
+    for i in range(args.warmup):
+        step(i)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    nbytes = sum(sum(step_bytes(wl, i % nsteps)) for i in range(args.steps))
+    world = 1 if not torch.distributed.is_initialized() else torch.distributed.get_world_size()
+    return {"value": world * nbytes / (ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms / args.steps,
+            "tokens_per_s": world * args.steps * wl.B / (ms * 1e-3)}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return reference_arm(args, rank, world)
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return npv_arm(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,335 @@
+// libnpv: the C ABI declared in include/npv.h.
+//
+// One translation unit: the kernels are included here so that the library-wide
+// device error word is a single symbol without relocatable device code.
+// Host functions validate every argument before launching, translate CUDA
+// errors into npv_status codes and never throw.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "npv.h"
+#include "npv_device.cuh"
+#include "store_kvcache.cuh"
+#include "decode_attention.cuh"
+
+#define NPV_VERSION_MAJOR 0
+#define NPV_VERSION_MINOR 1
+#define NPV_VERSION_PATCH 0
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    int sm_count = 0;
+    int max_smem_optin = 0;
+};
+
+DeviceInfo g_devices[kMaxDevices];
+std::once_flag g_device_once[kMaxDevices];
+
+// Properties of the current device (queried once per device).
+const DeviceInfo *current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::call_once(g_device_once[dev], [dev] {
+        DeviceInfo info;
+        cudaDeviceGetAttribute(&info.sm_count, cudaDevAttrMultiProcessorCount, dev);
+        cudaDeviceGetAttribute(&info.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        g_devices[dev] = info;
+    });
+    return g_devices[dev].sm_count > 0 ? &g_devices[dev] : nullptr;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+npv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NPV_OK : NPV_ERR_CUDA; }
+
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// while the previous kernel on the stream drains; every kernel of this library
+// calls griddepcontrol.wait before touching memory, so ordering is preserved.
+template <typename Kernel, typename... Args>
+cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// ---- decode configuration ------------------------------------------------------
+
+struct DecodeConfig {
+    int group = 0;           // g = Hq / Hkv
+    int heads_per_cta = 0;   // HC
+    int head_groups = 0;     // Hkv / HC
+    int stages = 0;
+    int grid = 0;
+    size_t smem = 0;
+    size_t ws_meta = 0, ws_ml = 0, ws_o = 0, ws_total = 0;
+};
+
+bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
+
+// Largest divisor of Hkv that is at most 8 (one consumer warp per KV head).
+int pick_heads_per_cta(int num_kv_heads) {
+    for (int hc = 8; hc >= 1; --hc)
+        if (num_kv_heads % hc == 0) return hc;
+    return 1;
+}
+
+npv_status decode_config(int num_q_heads, int num_kv_heads, int head_dim, DecodeConfig *cfg) {
+    if (num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return NPV_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return NPV_ERR_UNSUPPORTED;
+    const int g = num_q_heads / num_kv_heads;
+    if (!supported_group(g)) return NPV_ERR_UNSUPPORTED;
+    const DeviceInfo *dev = current_device();
+    if (!dev) return NPV_ERR_CUDA;
+    cfg->group = g;
+    cfg->heads_per_cta = pick_heads_per_cta(num_kv_heads);
+    cfg->head_groups = num_kv_heads / cfg->heads_per_cta;
+    const int hc = cfg->heads_per_cta;
+    const size_t stage_bytes = 2ull * npv::decode::kChunk * hc * head_dim * 2;
+    int stages = (int)(npv::decode::kStageBudgetBytes / stage_bytes);
+    if (stages > npv::decode::kMaxStages) stages = npv::decode::kMaxStages;
+    if (stages < 2) stages = 2;
+    cfg->stages = stages;
+    const size_t pbuf = align_up((size_t)hc * npv::decode::kChunk * g * 4, 1024);
+    cfg->smem = npv::decode::kHeaderBytes + pbuf + stages * stage_bytes;
+    if ((int)cfg->smem > dev->max_smem_optin) return NPV_ERR_UNSUPPORTED;
+    cfg->grid = dev->sm_count;
+    const size_t hcg = (size_t)hc * g;
+    cfg->ws_meta = align_up((size_t)cfg->grid * 4 * sizeof(long long), 256);
+    cfg->ws_ml = align_up((size_t)cfg->grid * 2 * hcg * sizeof(float2), 256);
+    cfg->ws_o = align_up((size_t)cfg->grid * 2 * hcg * head_dim * sizeof(float), 256);
+    cfg->ws_total = cfg->ws_meta + cfg->ws_ml + cfg->ws_o;
+    return NPV_OK;
+}
+
+template <int D, int G>
+cudaError_t launch_decode_split(const npv::decode::Params &p, const DecodeConfig &cfg, cudaStream_t stream) {
+    auto kernel = npv::decode::decode_split_kernel<D, G>;
+    static int configured_smem[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < kMaxDevices && configured_smem[dev] < (int)cfg.smem) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cfg.smem);
+        if (e != cudaSuccess) return e;
+        configured_smem[dev] = (int)cfg.smem;
+    }
+    return launch_pdl(kernel, dim3(cfg.grid), dim3((cfg.heads_per_cta + 1) * 32), cfg.smem, stream, p);
+}
+
+cudaError_t dispatch_decode_split(int D, const npv::decode::Params &p, const DecodeConfig &cfg,
+                                  cudaStream_t stream) {
+#define NPV_DECODE_CASE(DD, GG) \
+    if (D == DD && cfg.group == GG) return launch_decode_split<DD, GG>(p, cfg, stream);
+    NPV_DECODE_CASE(128, 1)
+    NPV_DECODE_CASE(128, 2)
+    NPV_DECODE_CASE(128, 4)
+    NPV_DECODE_CASE(128, 8)
+    NPV_DECODE_CASE(64, 1)
+    NPV_DECODE_CASE(64, 2)
+    NPV_DECODE_CASE(64, 4)
+    NPV_DECODE_CASE(64, 8)
+#undef NPV_DECODE_CASE
+    return cudaErrorInvalidValue;
+}
+
+// Shared by the decode call and the decode rows of the prefill call.
+npv_status run_decode(void *out, const void *q, int64_t q_row_stride, const int32_t *cu_seqlens_q,
+                      const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                      int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs,
+                      int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks,
+                      int32_t block_size, float scale, void *workspace, const DecodeConfig &cfg,
+                      cudaStream_t stream) {
+    npv::decode::Params p = {};
+    p.out = static_cast<uint16_t *>(out);
+    p.q = static_cast<const uint16_t *>(q);
+    p.q_row_stride = q_row_stride;
+    p.k_cache = static_cast<const uint16_t *>(k_cache);
+    p.v_cache = static_cast<const uint16_t *>(v_cache);
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.cu_seqlens_q = cu_seqlens_q;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_seqs = num_seqs;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.num_blocks = num_blocks;
+    p.block_size = block_size;
+    p.heads_per_cta = cfg.heads_per_cta;
+    p.num_head_groups = cfg.head_groups;
+    p.num_stages = cfg.stages;
+    const float s = scale > 0.f ? scale : (float)(1.0 / std::sqrt((double)head_dim));
+    p.scale_log2 = s * 1.4426950408889634f;
+    char *ws = static_cast<char *>(workspace);
+    p.meta = reinterpret_cast<long long *>(ws);
+    p.part_ml = reinterpret_cast<float2 *>(ws + cfg.ws_meta);
+    p.part_o = reinterpret_cast<float *>(ws + cfg.ws_meta + cfg.ws_ml);
+    cudaError_t e = dispatch_decode_split(head_dim, p, cfg, stream);
+    if (e != cudaSuccess) return NPV_ERR_CUDA;
+    e = launch_pdl(npv::decode::decode_merge_kernel, dim3(cfg.grid), dim3(256), 0, stream, p, (int)head_dim);
+    return cuda_status(e);
+}
+
+bool cache_shape_ok(int32_t num_blocks, int32_t block_size, int32_t num_kv_heads, int32_t head_dim) {
+    return num_blocks > 0 && block_size > 0 && num_kv_heads > 0 && head_dim > 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *npv_status_string(npv_status status) {
+    switch (status) {
+        case NPV_OK: return "ok";
+        case NPV_ERR_INVALID_ARG: return "invalid argument (null pointer, bad shape, misaligned pointer or stride)";
+        case NPV_ERR_UNSUPPORTED: return "unsupported configuration";
+        case NPV_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case NPV_ERR_CUDA: return "CUDA runtime error";
+        case NPV_ERR_DEVICE_BOUNDS: return "device reported an out-of-range slot, block id or length";
+    }
+    return "unknown status";
+}
+
+int npv_version(void) { return NPV_VERSION_MAJOR * 10000 + NPV_VERSION_MINOR * 100 + NPV_VERSION_PATCH; }
+
+npv_status npv_store_kvcache(const void *key, const void *value, int64_t key_token_stride,
+                             int64_t value_token_stride, void *k_cache, void *v_cache,
+                             const int32_t *slot_mapping, int32_t num_tokens, int32_t num_blocks,
+                             int32_t block_size, int32_t num_kv_heads, int32_t head_dim, npv_stream_t stream) {
+    if (num_tokens < 0 || !cache_shape_ok(num_blocks, block_size, num_kv_heads, head_dim))
+        return NPV_ERR_INVALID_ARG;
+    if (num_tokens == 0) return NPV_OK;
+    if (!key || !value || !k_cache || !v_cache || !slot_mapping) return NPV_ERR_INVALID_ARG;
+    const int64_t row = (int64_t)num_kv_heads * head_dim;
+    if (key_token_stride == 0) key_token_stride = row;
+    if (value_token_stride == 0) value_token_stride = row;
+    if (key_token_stride < row || value_token_stride < row) return NPV_ERR_INVALID_ARG;
+    if ((row * 2) % 16 != 0 || (key_token_stride * 2) % 16 != 0 || (value_token_stride * 2) % 16 != 0)
+        return NPV_ERR_INVALID_ARG;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache))
+        return NPV_ERR_INVALID_ARG;
+    const DeviceInfo *dev = current_device();
+    if (!dev) return NPV_ERR_CUDA;
+    npv::store::Params p = {};
+    p.key = static_cast<const uint16_t *>(key);
+    p.value = static_cast<const uint16_t *>(value);
+    p.key_stride = key_token_stride;
+    p.value_stride = value_token_stride;
+    p.k_cache = static_cast<uint16_t *>(k_cache);
+    p.v_cache = static_cast<uint16_t *>(v_cache);
+    p.slot_mapping = slot_mapping;
+    p.num_tokens = num_tokens;
+    p.row_vecs = (int32_t)(row / 8);
+    p.num_slots = (int64_t)num_blocks * block_size;
+    const int64_t vecs = (int64_t)num_tokens * p.row_vecs;
+    const int64_t per_block = (int64_t)npv::store::kThreads * npv::store::kVecsPerThread;
+    int64_t blocks = (vecs + per_block - 1) / per_block;
+    const int64_t cap = (int64_t)dev->sm_count * 8;
+    if (blocks > cap) blocks = cap;
+    cudaError_t e = launch_pdl(npv::store::store_kvcache_kernel, dim3((unsigned)blocks),
+                               dim3(npv::store::kThreads), 0, (cudaStream_t)stream, p);
+    return cuda_status(e);
+}
+
+size_t npv_paged_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                       int32_t head_dim) {
+    if (num_seqs < 0) return 0;
+    DecodeConfig cfg;
+    if (decode_config(num_q_heads, num_kv_heads, head_dim, &cfg) != NPV_OK) return 0;
+    return cfg.ws_total;
+}
+
+npv_status npv_paged_decode_attention(void *out, const void *q, int64_t q_seq_stride, const void *k_cache,
+                                      const void *v_cache, const int32_t *block_tables,
+                                      int32_t max_blocks_per_seq, const int32_t *context_lens,
+                                      int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                      int32_t head_dim, int32_t num_blocks, int32_t block_size, float scale,
+                                      void *workspace, size_t workspace_bytes, npv_stream_t stream) {
+    if (num_seqs < 0 || max_blocks_per_seq <= 0 || !cache_shape_ok(num_blocks, block_size, num_kv_heads, head_dim))
+        return NPV_ERR_INVALID_ARG;
+    if (num_q_heads <= 0 || num_q_heads % num_kv_heads != 0) return NPV_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return NPV_ERR_INVALID_ARG;
+    if (block_size % 16 != 0) return NPV_ERR_UNSUPPORTED;
+    DecodeConfig cfg;
+    npv_status st = decode_config(num_q_heads, num_kv_heads, head_dim, &cfg);
+    if (st != NPV_OK) return st;
+    if (num_seqs == 0) return NPV_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return NPV_ERR_INVALID_ARG;
+    const int64_t qrow = (int64_t)num_q_heads * head_dim;
+    if (q_seq_stride == 0) q_seq_stride = qrow;
+    if (q_seq_stride < qrow || (q_seq_stride * 2) % 16 != 0) return NPV_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return NPV_ERR_INVALID_ARG;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < cfg.ws_total)
+        return NPV_ERR_WORKSPACE;
+    return run_decode(out, q, q_seq_stride, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                      context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, scale,
+                      workspace, cfg, (cudaStream_t)stream);
+}
+
+size_t npv_paged_prefill_workspace_size(int32_t num_seqs, int32_t total_q, int32_t num_q_heads,
+                                        int32_t num_kv_heads, int32_t head_dim) {
+    (void)num_seqs;
+    (void)total_q;
+    (void)num_q_heads;
+    (void)num_kv_heads;
+    (void)head_dim;
+    return 0;
+}
+
+npv_status npv_paged_prefill_attention(void *out, const void *q, const int32_t *cu_seqlens_q,
+                                       int32_t max_seqlen_q, int32_t total_q, const void *k_cache,
+                                       const void *v_cache, const int32_t *block_tables,
+                                       int32_t max_blocks_per_seq, const int32_t *context_lens,
+                                       int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                       int32_t head_dim, int32_t num_blocks, int32_t block_size, float scale,
+                                       void *workspace, size_t workspace_bytes, npv_stream_t stream) {
+    (void)out;
+    (void)q;
+    (void)cu_seqlens_q;
+    (void)max_seqlen_q;
+    (void)total_q;
+    (void)k_cache;
+    (void)v_cache;
+    (void)block_tables;
+    (void)max_blocks_per_seq;
+    (void)context_lens;
+    (void)num_seqs;
+    (void)num_q_heads;
+    (void)num_kv_heads;
+    (void)head_dim;
+    (void)num_blocks;
+    (void)block_size;
+    (void)scale;
+    (void)workspace;
+    (void)workspace_bytes;
+    (void)stream;
+    return NPV_ERR_UNSUPPORTED;
+}
+
+npv_status npv_check_device_errors(npv_stream_t stream, uint32_t *bits_out) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return NPV_ERR_CUDA;
+    unsigned int bits = 0;
+    if (cudaMemcpyFromSymbol(&bits, npv::g_error_word, sizeof(bits)) != cudaSuccess) return NPV_ERR_CUDA;
+    if (bits != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(npv::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return NPV_ERR_CUDA;
+    }
+    if (bits_out) *bits_out = bits;
+    return bits ? NPV_ERR_DEVICE_BOUNDS : NPV_OK;
+}
+
+}  // extern "C"

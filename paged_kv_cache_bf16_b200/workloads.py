@@ -436,3 +436,72 @@ def scaled(spec: Spec, **changes) -> Spec:
     d = dict(spec.__dict__)
     d.update(changes)
     return Spec(**d)
+
+
+# ---------------------------------------------------------------------------
+# Device copies (torch supplies the memory; nothing here computes attention)
+# ---------------------------------------------------------------------------
+
+def bits_to_torch(a: np.ndarray, device=None):
+    """uint16 bf16 bit patterns -> torch.bfloat16 tensor (same bits)."""
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+    return t.to(device) if device is not None else t
+
+
+def torch_to_bits(t) -> np.ndarray:
+    """torch.bfloat16 tensor -> uint16 numpy array of its bit patterns."""
+    import torch
+
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+class DeviceState:
+    """A workload's cache and per-step inputs resident on one CUDA device.
+
+    The caches are [NB, BS, Hkv, D] bf16, filled with bf16 NaN except the cached
+    prefix of every sequence, so any read outside a sequence's live tokens shows
+    up as NaN in the output.
+    """
+
+    def __init__(self, wl: Workload, device, steps: Optional[List[int]] = None):
+        import torch
+
+        self.wl = wl
+        self.device = torch.device(device)
+        shape = (wl.NB, wl.BS, wl.Hkv, wl.D)
+        self.k_cache = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
+        self.v_cache = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
+        nan = int(np.int16(np.uint16(BF16_NAN).view(np.int16)))
+        self.k_cache.view(torch.int16).fill_(nan)
+        self.v_cache.view(torch.int16).fill_(nan)
+        ids, K, V = wl.prior_blocks_dense()
+        if len(ids):
+            idx = torch.from_numpy(ids).to(self.device)
+            # copy in slices to bound the host->device staging footprint
+            step = max(1, (1 << 28) // max(1, K[0].nbytes))
+            for s in range(0, len(ids), step):
+                self.k_cache.index_copy_(0, idx[s:s + step], bits_to_torch(K[s:s + step], self.device))
+                self.v_cache.index_copy_(0, idx[s:s + step], bits_to_torch(V[s:s + step], self.device))
+        del K, V
+        self.steps = {}
+        for st in (steps if steps is not None else [0]):
+            self.steps[st] = self.step_inputs(st)
+
+    def step_inputs(self, step: int) -> Dict[str, "object"]:
+        import torch
+
+        wl = self.wl
+        d = self.device
+        k, v = wl.new_kv(step)
+        return {
+            "q": bits_to_torch(wl.q(step), d),
+            "key": bits_to_torch(k, d),
+            "value": bits_to_torch(v, d),
+            "slot_mapping": torch.from_numpy(wl.slot_mapping(step)).to(d),
+            "block_tables": torch.from_numpy(wl.block_tables(step)).to(d),
+            "context_lens": torch.from_numpy(wl.context_lens(step)).to(d),
+            "cu_seqlens_q": torch.from_numpy(wl.cu_seqlens_q()).to(d),
+            "max_seqlen_q": int(wl.query_lens.max()) if wl.B else 0,
+        }

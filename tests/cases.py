@@ -35,42 +35,50 @@ def oracle_attention(wl: W.Workload, kp: np.ndarray, vp: np.ndarray, step: int =
                              wl.cu_seqlens_q(), scale=scale, threads=threads, _lib=lib)
 
 
-def compact_seq_pool(wl: W.Workload, b: int, step: int, kp_full=None, vp_full=None):
-    """The blocks of sequence b (after stores up to `step`) relabelled 0..n-1.
+def oracle_compact(wl: W.Workload, step: int = 0, seqs=None, lib=None, threads: Optional[int] = None,
+                   scale: float = 0.0):
+    """Oracle outputs for sequences `seqs` (default: all) at `step`.
 
-    Physical relabelling leaves attention unchanged (a pinned oracle property),
-    so a compact pool stands in for a 4,096- or 57,344-block pool when the
-    oracle checks sampled sequences of a full-size workload.
-    Returns (k_pool, v_pool, block_table_row, context_len).
+    The oracle gets a pool holding only the blocks those sequences reference,
+    relabelled 0..n-1 in order of first use (relabelling is a pinned invariant),
+    the cached prefixes, and every store of steps 0..step applied by the
+    oracle's own store.  Returns (fp64 out [rows, Hq, D], packed row indices).
     """
-    L = int(wl.context_lens(step)[b])
-    nblk = -(-L // wl.BS)
-    blocks = [int(p) for p in wl.seq_blocks[b][:nblk]]
-    shape = (nblk, wl.BS, wl.Hkv, wl.D)
+    from oracle import oracle as O
+
+    seqs = list(range(wl.B)) if seqs is None else [int(b) for b in seqs]
+    L = wl.context_lens(step)
+    bt = wl.block_tables(step)
+    remap = {}
+    bt_c = np.full((len(seqs), wl.max_blocks_per_seq), -1, dtype=np.int32)
+    for r, b in enumerate(seqs):
+        for i in range(-(-int(L[b]) // wl.BS)):
+            p = int(bt[b, i])
+            if p not in remap:
+                remap[p] = len(remap)
+            bt_c[r, i] = remap[p]
+    n = max(1, len(remap))
+    shape = (n, wl.BS, wl.Hkv, wl.D)
     kp = np.full(shape, W.BF16_NAN, dtype=np.uint16)
     vp = np.full(shape, W.BF16_NAN, dtype=np.uint16)
-    if kp_full is not None:
-        kp[:] = kp_full[blocks]
-        vp[:] = vp_full[blocks]
-        return kp, vp, np.arange(nblk, dtype=np.int32), L
-    # cached prefix from the generator, then every new token stored up to `step`
-    pl = wl.prior_len(b)
-    for i, p in enumerate(blocks):
-        n = max(0, min(wl.BS, pl - i * wl.BS))
-        if n:
-            k, v = wl.block_contents(p, n)
-            kp[i, :n] = k
-            vp[i, :n] = v
-    hd = wl.Hkv * wl.D
-    j0 = pl
-    n_new = L - pl
-    if n_new > 0:
-        k = W.normal_bf16(W.stream_key(wl.spec.seed, W.TAG_NEW_K, b), j0 * hd, n_new * hd, wl.spec.sigma)
-        v = W.normal_bf16(W.stream_key(wl.spec.seed, W.TAG_NEW_V, b), j0 * hd, n_new * hd, wl.spec.sigma)
-        k = k.reshape(n_new, wl.Hkv, wl.D)
-        v = v.reshape(n_new, wl.Hkv, wl.D)
-        for t in range(n_new):
-            j = j0 + t
-            kp[j // wl.BS, j % wl.BS] = k[t]
-            vp[j // wl.BS, j % wl.BS] = v[t]
-    return kp, vp, np.arange(nblk, dtype=np.int32), L
+    for p, nv in wl.prior_fill():
+        if p in remap:
+            k, v = wl.block_contents(p, nv)
+            kp[remap[p], :nv] = k
+            vp[remap[p], :nv] = v
+    chosen = np.zeros(wl.B, dtype=bool)
+    chosen[seqs] = True
+    for s in range(step + 1):
+        seq_of_tok, _ = wl.token_positions(s)
+        keep = chosen[seq_of_tok]
+        slots = wl.slot_mapping(s)[keep]
+        k, v = wl.new_kv(s)
+        cslots = np.array([remap[int(x) // wl.BS] * wl.BS + int(x) % wl.BS for x in slots], dtype=np.int32)
+        O.store_kvcache(k[keep], v[keep], kp, vp, cslots, _lib=lib)
+    cu = wl.cu_seqlens_q()
+    rows = np.concatenate([np.arange(cu[b], cu[b + 1]) for b in seqs]) if seqs else np.zeros(0, np.int64)
+    qsub = wl.q(step)[rows]
+    cu_c = np.zeros(len(seqs) + 1, dtype=np.int32)
+    cu_c[1:] = np.cumsum(wl.query_lens[seqs])
+    out = O.paged_attention(qsub, kp, vp, bt_c, L[seqs], cu_c, scale=scale, threads=threads, _lib=lib)
+    return out, rows
