@@ -426,9 +426,23 @@ SPECS: Dict[str, Spec] = {
 # Headline workload for throughput reporting.
 HEADLINE = "qwen3_decode"
 
+# Smaller variants of the same shapes, for profiler captures that must stay a
+# few GB on the device (the KV read per launch still exceeds the 126 MB L2).
+PROFILE_SPECS: Dict[str, Spec] = {
+    "qwen3_decode_small": Spec(
+        name="qwen3_decode_small", seed=2, num_seqs=64, num_q_heads=16, num_kv_heads=8, head_dim=128,
+        block_size=256, num_blocks=1024, ctx_lo=100, ctx_hi=2048, num_steps=4,
+        description="qwen3_decode with 64 sequences and a 1,024-block pool (profiling size)"),
+    "chunked_prefill_small": Spec(
+        name="chunked_prefill_small", seed=5, num_seqs=68, num_q_heads=16, num_kv_heads=8, head_dim=128,
+        block_size=256, num_blocks=1024, ctx_lo=100, ctx_hi=2048, prefill_seqs=4, prefill_len=512,
+        prior_lo=0, prior_hi=8192,
+        description="chunked_prefill_mixed with 4 prefill + 64 decode sequences (profiling size)"),
+}
+
 
 def workload(name: str) -> Workload:
-    return draw(SPECS[name])
+    return draw(SPECS[name] if name in SPECS else PROFILE_SPECS[name])
 
 
 def scaled(spec: Spec, **changes) -> Spec:
