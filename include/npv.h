@@ -186,6 +186,40 @@ NPV_API npv_status npv_paged_prefill_attention(void *out, const void *q, const i
                                        int32_t head_dim, int32_t num_blocks, int32_t block_size, float scale,
                                        void *workspace, size_t workspace_bytes, npv_stream_t stream);
 
+/* Size of the scratch array compiled into the library for
+ * npv_paged_decode_attention_noalloc (16 MiB on every device that loads it). */
+#define NPV_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/*
+ * Decode attention for callers that cannot allocate device memory.  The pages
+ * have no counterpart to this entry point; it is a convenience of this library.
+ *
+ * Some callers cannot call cudaMalloc or hand the library a workspace: a plugin
+ * or custom-op host whose framework owns all device memory and passes only its
+ * input and output buffers, or code on a path where an allocation is not
+ * allowed because cudaMalloc may synchronise the device.  This call computes
+ * exactly what npv_paged_decode_attention computes (same arguments, minus the
+ * workspace) and allocates nothing: its scratch is a fixed array of
+ * NPV_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ * library holds until the process exits.
+ *   - The first call on each device looks up that array's device address (a
+ *     one-time set-up that may load the library's GPU code).  Make the first
+ *     call on a device before any stream capture begins.
+ *   - A head configuration whose scratch would not fit returns
+ *     NPV_ERR_WORKSPACE (on a 148-SM B200 every supported configuration fits).
+ *   - All calls share the one array, which keeps whatever the last call left in
+ *     it; nothing in it needs to start at zero.  Calls that overlap on the GPU
+ *     (on different streams, or from several host threads at once) race on it
+ *     and produce wrong results; calls ordered on one stream are safe.
+ */
+NPV_API npv_status npv_paged_decode_attention_noalloc(void *out, const void *q, int64_t q_seq_stride,
+                                                      const void *k_cache, const void *v_cache,
+                                                      const int32_t *block_tables, int32_t max_blocks_per_seq,
+                                                      const int32_t *context_lens, int32_t num_seqs,
+                                                      int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                                      int32_t num_blocks, int32_t block_size, float scale,
+                                                      npv_stream_t stream);
+
 /*
  * Synchronise `stream`, then read and clear the device error word of the
  * current device.  Returns NPV_OK if no error was recorded since the last

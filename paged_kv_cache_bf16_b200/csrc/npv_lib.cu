@@ -333,3 +333,6 @@ npv_status npv_check_device_errors(npv_stream_t stream, uint32_t *bits_out) {
 }
 
 }  // extern "C"
+
+// The allocation-free decode entry point shares this translation unit.
+#include "npv_noalloc.cu"
