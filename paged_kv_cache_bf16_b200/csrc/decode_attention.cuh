@@ -59,6 +59,7 @@ struct Params {
     const int32_t *block_tables;
     const int32_t *context_lens;
     const int32_t *cu_seqlens_q;  // non-null: mixed batch; only sequences with one query row run here
+    int32_t total_q;              // rows of q and out in a mixed batch
     int32_t max_blocks_per_seq;
     int32_t num_seqs;
     int32_t num_q_heads;
@@ -80,8 +81,8 @@ struct Params {
 __device__ __forceinline__ int32_t seq_chunks(const Params &p, int32_t b) {
     const int32_t L = __ldg(p.context_lens + b);
     if (p.cu_seqlens_q != nullptr) {
-        const int32_t n = __ldg(p.cu_seqlens_q + b + 1) - __ldg(p.cu_seqlens_q + b);
-        if (n != 1) return 0;
+        const int32_t cb = __ldg(p.cu_seqlens_q + b), ce = __ldg(p.cu_seqlens_q + b + 1);
+        if (ce - cb != 1 || cb < 0 || ce > p.total_q) return 0;
     }
     if (L <= 0 || (long long)L > (long long)p.max_blocks_per_seq * p.block_size) return 0;
     return (L + kChunk - 1) / kChunk;
@@ -488,9 +489,12 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const Params p, int h
     // (1) rows with no chunks on this path
     for (long long b = c + (long long)G * threadIdx.x; b < p.num_seqs; b += G * blockDim.x) {
         const int32_t L = __ldg(p.context_lens + b);
-        int32_t n = 1;
-        if (p.cu_seqlens_q != nullptr) n = __ldg(p.cu_seqlens_q + b + 1) - __ldg(p.cu_seqlens_q + b);
-        if (n != 1) continue;  // multi-row sequences belong to the prefill kernel
+        if (p.cu_seqlens_q != nullptr) {
+            const int32_t cb = __ldg(p.cu_seqlens_q + b), ce = __ldg(p.cu_seqlens_q + b + 1);
+            // multi-row sequences belong to the prefill kernel, which also
+            // reports malformed cu_seqlens_q
+            if (ce - cb != 1 || cb < 0 || ce > p.total_q) continue;
+        }
         const bool bad = L < 0 || (long long)L > (long long)p.max_blocks_per_seq * p.block_size ||
                          (p.cu_seqlens_q != nullptr && L < 1);
         if (bad) report_error(NPV_DEVERR_CONTEXT_LEN);

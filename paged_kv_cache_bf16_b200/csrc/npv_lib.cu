@@ -4,6 +4,7 @@
 // device error word is a single symbol without relocatable device code.
 // Host functions validate every argument before launching, translate CUDA
 // errors into npv_status codes and never throw.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -14,6 +15,7 @@
 #include "npv_device.cuh"
 #include "store_kvcache.cuh"
 #include "decode_attention.cuh"
+#include "prefill_attention.cuh"
 
 #define NPV_VERSION_MAJOR 0
 #define NPV_VERSION_MINOR 1
@@ -148,7 +150,7 @@ cudaError_t dispatch_decode_split(int D, const npv::decode::Params &p, const Dec
 }
 
 // Shared by the decode call and the decode rows of the prefill call.
-npv_status run_decode(void *out, const void *q, int64_t q_row_stride, const int32_t *cu_seqlens_q,
+npv_status run_decode(void *out, const void *q, int64_t q_row_stride, const int32_t *cu_seqlens_q, int32_t total_q,
                       const void *k_cache, const void *v_cache, const int32_t *block_tables,
                       int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs,
                       int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks,
@@ -163,6 +165,7 @@ npv_status run_decode(void *out, const void *q, int64_t q_row_stride, const int3
     p.block_tables = block_tables;
     p.context_lens = context_lens;
     p.cu_seqlens_q = cu_seqlens_q;
+    p.total_q = total_q;
     p.max_blocks_per_seq = max_blocks_per_seq;
     p.num_seqs = num_seqs;
     p.num_q_heads = num_q_heads;
@@ -182,6 +185,100 @@ npv_status run_decode(void *out, const void *q, int64_t q_row_stride, const int3
     if (e != cudaSuccess) return NPV_ERR_CUDA;
     e = launch_pdl(npv::decode::decode_merge_kernel, dim3(cfg.grid), dim3(256), 0, stream, p, (int)head_dim);
     return cuda_status(e);
+}
+
+// ---- prefill configuration ----------------------------------------------------
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled from the driver, found through the runtime (no libcuda link).
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 3-D bf16 tensor [d2][d1][d0] (d0 contiguous), 128-byte swizzled boxes of b0 x b1 x b2.
+bool encode_map_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
+                   uint32_t b1, uint32_t b2) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    const cuuint32_t box[3] = {b0, b1, b2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct PrefillConfig {
+    DecodeConfig decode;  // for the rows of single-row sequences
+    int32_t max_pairs = 0;
+    int grid = 0;
+    size_t smem = 0;
+    size_t ws_total = 0;
+};
+
+npv_status prefill_config(int32_t num_seqs, int32_t total_q, int num_q_heads, int num_kv_heads, int head_dim,
+                          PrefillConfig *cfg) {
+    if (num_seqs < 0 || total_q < 0) return NPV_ERR_INVALID_ARG;
+    npv_status st = decode_config(num_q_heads, num_kv_heads, head_dim, &cfg->decode);
+    if (st != NPV_OK) return st;
+    const DeviceInfo *dev = current_device();
+    if (!dev) return NPV_ERR_CUDA;
+    const int ppt = npv::prefill::kTileM / cfg->decode.group;
+    const int64_t pairs = (int64_t)total_q / ppt + 1 + num_seqs;
+    if (pairs > 0x7FFFFFFF) return NPV_ERR_UNSUPPORTED;
+    cfg->max_pairs = (int32_t)pairs;
+    cfg->grid = dev->sm_count;
+    cfg->smem = (head_dim == 128 ? npv::prefill::Smem<128>::total : npv::prefill::Smem<64>::total) + 1024;
+    if ((int)cfg->smem > dev->max_smem_optin) return NPV_ERR_UNSUPPORTED;
+    cfg->ws_total = cfg->decode.ws_total + 256 + align_up((size_t)pairs * sizeof(int2), 256);
+    return NPV_OK;
+}
+
+template <int D, int G>
+cudaError_t launch_prefill(const npv::prefill::Params &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
+                           const CUtensorMap &vmap, const PrefillConfig &cfg, cudaStream_t stream) {
+    cudaError_t e = launch_pdl(npv::prefill::prefill_plan_kernel<G>, dim3(1), dim3(1024), 0, stream, p, D);
+    if (e != cudaSuccess) return e;
+    auto kernel = npv::prefill::prefill_attention_kernel<D, G>;
+    static int configured_smem[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < kMaxDevices && configured_smem[dev] < (int)cfg.smem) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cfg.smem);
+        if (e != cudaSuccess) return e;
+        configured_smem[dev] = (int)cfg.smem;
+    }
+    return launch_pdl(kernel, dim3(cfg.grid), dim3(npv::prefill::kThreads), cfg.smem, stream, p, qmap, kmap, vmap);
+}
+
+cudaError_t dispatch_prefill(int D, int G, const npv::prefill::Params &p, const CUtensorMap &qmap,
+                             const CUtensorMap &kmap, const CUtensorMap &vmap, const PrefillConfig &cfg,
+                             cudaStream_t stream) {
+#define NPV_PREFILL_CASE(DD, GG) \
+    if (D == DD && G == GG) return launch_prefill<DD, GG>(p, qmap, kmap, vmap, cfg, stream);
+    NPV_PREFILL_CASE(128, 1)
+    NPV_PREFILL_CASE(128, 2)
+    NPV_PREFILL_CASE(128, 4)
+    NPV_PREFILL_CASE(128, 8)
+    NPV_PREFILL_CASE(64, 1)
+    NPV_PREFILL_CASE(64, 2)
+    NPV_PREFILL_CASE(64, 4)
+    NPV_PREFILL_CASE(64, 8)
+#undef NPV_PREFILL_CASE
+    return cudaErrorInvalidValue;
 }
 
 bool cache_shape_ok(int32_t num_blocks, int32_t block_size, int32_t num_kv_heads, int32_t head_dim) {
@@ -275,19 +372,16 @@ npv_status npv_paged_decode_attention(void *out, const void *q, int64_t q_seq_st
     if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return NPV_ERR_INVALID_ARG;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < cfg.ws_total)
         return NPV_ERR_WORKSPACE;
-    return run_decode(out, q, q_seq_stride, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq,
+    return run_decode(out, q, q_seq_stride, nullptr, num_seqs, k_cache, v_cache, block_tables, max_blocks_per_seq,
                       context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, scale,
                       workspace, cfg, (cudaStream_t)stream);
 }
 
 size_t npv_paged_prefill_workspace_size(int32_t num_seqs, int32_t total_q, int32_t num_q_heads,
                                         int32_t num_kv_heads, int32_t head_dim) {
-    (void)num_seqs;
-    (void)total_q;
-    (void)num_q_heads;
-    (void)num_kv_heads;
-    (void)head_dim;
-    return 0;
+    PrefillConfig cfg;
+    if (prefill_config(num_seqs, total_q, num_q_heads, num_kv_heads, head_dim, &cfg) != NPV_OK) return 0;
+    return cfg.ws_total;
 }
 
 npv_status npv_paged_prefill_attention(void *out, const void *q, const int32_t *cu_seqlens_q,
@@ -297,27 +391,59 @@ npv_status npv_paged_prefill_attention(void *out, const void *q, const int32_t *
                                        int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
                                        int32_t head_dim, int32_t num_blocks, int32_t block_size, float scale,
                                        void *workspace, size_t workspace_bytes, npv_stream_t stream) {
-    (void)out;
-    (void)q;
-    (void)cu_seqlens_q;
-    (void)max_seqlen_q;
-    (void)total_q;
-    (void)k_cache;
-    (void)v_cache;
-    (void)block_tables;
-    (void)max_blocks_per_seq;
-    (void)context_lens;
-    (void)num_seqs;
-    (void)num_q_heads;
-    (void)num_kv_heads;
-    (void)head_dim;
-    (void)num_blocks;
-    (void)block_size;
-    (void)scale;
-    (void)workspace;
-    (void)workspace_bytes;
-    (void)stream;
-    return NPV_ERR_UNSUPPORTED;
+    if (num_seqs < 0 || total_q < 0 || max_seqlen_q < 0 || max_blocks_per_seq <= 0 ||
+        !cache_shape_ok(num_blocks, block_size, num_kv_heads, head_dim))
+        return NPV_ERR_INVALID_ARG;
+    if (num_q_heads <= 0 || num_q_heads % num_kv_heads != 0) return NPV_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return NPV_ERR_INVALID_ARG;
+    if (block_size % 16 != 0) return NPV_ERR_UNSUPPORTED;
+    if ((int64_t)num_blocks * block_size > 0xFFFFFFFFll) return NPV_ERR_UNSUPPORTED;
+    PrefillConfig cfg;
+    npv_status st = prefill_config(num_seqs, total_q, num_q_heads, num_kv_heads, head_dim, &cfg);
+    if (st != NPV_OK) return st;
+    if (num_seqs == 0 || total_q == 0) return NPV_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !cu_seqlens_q)
+        return NPV_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return NPV_ERR_INVALID_ARG;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < cfg.ws_total)
+        return NPV_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int D = head_dim, G = cfg.decode.group;
+
+    // tensor maps: q [total_q, Hq, D] and the caches [NB * BS, Hkv, D], 128-byte swizzle
+    CUtensorMap qmap, kmap, vmap;
+    const int box_tokens = (block_size % 128 == 0) ? 128 : 16;
+    if (!encode_map_3d(&qmap, q, D, num_q_heads, total_q, 64, G, 128 / G) ||
+        !encode_map_3d(&kmap, k_cache, D, num_kv_heads, (uint64_t)num_blocks * block_size, 64, 1, box_tokens) ||
+        !encode_map_3d(&vmap, v_cache, D, num_kv_heads, (uint64_t)num_blocks * block_size, 64, 1, box_tokens))
+        return NPV_ERR_CUDA;
+
+    npv::prefill::Params p = {};
+    p.out = static_cast<uint16_t *>(out);
+    p.cu_seqlens_q = cu_seqlens_q;
+    p.context_lens = context_lens;
+    p.block_tables = block_tables;
+    p.total_q = total_q;
+    p.num_seqs = num_seqs;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.num_blocks = num_blocks;
+    p.block_size = block_size;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.box_tokens = box_tokens;
+    const float sc = scale > 0.f ? scale : (float)(1.0 / std::sqrt((double)head_dim));
+    p.scale_log2 = sc * 1.4426950408889634f;
+    char *ws = static_cast<char *>(workspace);
+    p.plan_count = reinterpret_cast<int32_t *>(ws + cfg.decode.ws_total);
+    p.plan_pairs = reinterpret_cast<int2 *>(ws + cfg.decode.ws_total + 256);
+    p.max_pairs = cfg.max_pairs;
+
+    cudaError_t e = dispatch_prefill(D, G, p, qmap, kmap, vmap, cfg, s);
+    if (e != cudaSuccess) return NPV_ERR_CUDA;
+    // rows of sequences with exactly one query row: split-KV decode
+    return run_decode(out, q, (int64_t)num_q_heads * head_dim, cu_seqlens_q, total_q, k_cache, v_cache,
+                      block_tables, max_blocks_per_seq, context_lens, num_seqs, num_q_heads, num_kv_heads,
+                      head_dim, num_blocks, block_size, scale, workspace, cfg.decode, s);
 }
 
 npv_status npv_check_device_errors(npv_stream_t stream, uint32_t *bits_out) {

@@ -71,7 +71,7 @@ extern "C" NPV_API npv_status npv_paged_decode_attention_noalloc(
     if (st != NPV_OK) return st;
     // Nothing in the scratch has to start at zero: every slot the merge kernel
     // reads is written earlier in the same call by the split kernel.
-    return run_decode(out, q, q_seq_stride, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq,
+    return run_decode(out, q, q_seq_stride, nullptr, num_seqs, k_cache, v_cache, block_tables, max_blocks_per_seq,
                       context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, scale,
                       scratch, cfg, (cudaStream_t)stream);
 }
