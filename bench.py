@@ -38,6 +38,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "paged GQA decode attention: achieved HBM GB/s (% of peak), tokens/s"
+MIXED_METRIC = "chunked-prefill mixed batch attention: HBM GB/s, tokens/s, prefill TFLOP/s"
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 KERNEL_SRC = os.path.join(ROOT, "paged_kv_cache_bf16_b200", "csrc", "decode_attention.cuh")
@@ -52,6 +53,8 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="qwen3_decode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--separate-store", action="store_true",
+                    help="decode steps as npv_store_kvcache + npv_paged_decode_attention instead of the fused call")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline budget")
     ap.add_argument("--ref-seconds", type=float, default=150.0, help="reference-arm budget")
     return ap.parse_args(argv)
@@ -65,6 +68,16 @@ def measured_peaks():
         return float(d["hbm_gbs"]), "measured"
     except (OSError, KeyError, ValueError):
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_tflops():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured burst bf16 (MEASURED_PEAKS.json bf16_tflops)"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, "fallback 1590 TFLOP/s"
 
 
 def kernel_source_hash() -> str:
@@ -97,16 +110,33 @@ def profiled_traffic(workload: str):
 # workload bookkeeping (host side)
 # ---------------------------------------------------------------------------
 
-def step_bytes(wl, step):
-    """Algorithmic HBM bytes of one step: (store, decode attention)."""
+def step_bytes(wl, step, seqs=None):
+    """Algorithmic HBM bytes of one step over `seqs` (default all): (store, attention).
+
+    Attention reads each sequence's live K/V once, reads q, writes out and reads
+    the metadata; the store reads and writes each new K/V row once."""
+    seqs = np.arange(wl.B) if seqs is None else np.asarray(seqs)
     row = wl.Hkv * wl.D * 2
-    T = wl.total_q
-    store = 2 * T * row * 2  # read key+value rows, write them into the caches
+    nq = int(wl.query_lens[seqs].sum())
+    store = 2 * nq * row * 2
+    L = wl.context_lens(step).astype(np.int64)[seqs]
+    qo = 2 * nq * wl.Hq * wl.D * 2
+    meta = len(seqs) * 8 + int(sum(-(-int(x) // wl.BS) for x in L)) * 4
+    attn = int(L.sum()) * 2 * row + qo + meta
+    return store, attn
+
+
+def prefill_flops(wl, step=0, seqs=None):
+    """Algorithmic FLOPs of the attention of `seqs`: 4 * D per (query head, visible key) pair
+    (2 * D for q.k, 2 * D for p.v)."""
+    seqs = np.arange(wl.B) if seqs is None else np.asarray(seqs)
     L = wl.context_lens(step).astype(np.int64)
-    qo = 2 * wl.total_q * wl.Hq * wl.D * 2  # read q, write out
-    meta = wl.B * 4 + int(sum(-(-int(x) // wl.BS) for x in L)) * 4
-    decode = int(L.sum()) * 2 * row + qo + meta
-    return store, decode
+    total = 0
+    for b in seqs:
+        n = int(wl.query_lens[b])
+        prior = int(L[b]) - n
+        total += n * prior + n * (n + 1) // 2
+    return 4 * wl.D * wl.Hq * total
 
 
 class ClockSampler:
@@ -288,19 +318,36 @@ def npv_arm(args, rank, world, local_rank):
     ops.lib()
     wl = W.workload(args.workload)
     nsteps = wl.spec.num_steps
+    mixed = wl.spec.prefill_seqs > 0
     st = W.DeviceState(wl, dev, steps=list(range(nsteps)))
-    ws = ops.alloc_workspace(ops.decode_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.D), dev)
-    out = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device=dev)
+    if mixed:
+        ws = ops.alloc_workspace(ops.prefill_workspace_size(wl.B, wl.total_q, wl.Hq, wl.Hkv, wl.D), dev)
+        out = torch.empty((wl.total_q, wl.Hq, wl.D), dtype=torch.bfloat16, device=dev)
+    else:
+        ws = ops.alloc_workspace(ops.decode_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.D), dev)
+        out = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def store(i):
+    def attend(i):
         s = st.steps[i % nsteps]
-        ops.store_kvcache(s["key"], s["value"], st.k_cache, st.v_cache, s["slot_mapping"])
+        if mixed:
+            ops.paged_prefill_attention(s["q"], st.k_cache, st.v_cache, s["cu_seqlens_q"], s["max_seqlen_q"],
+                                        s["block_tables"], s["context_lens"], out=out, workspace=ws)
+        elif args.separate_store:
+            ops.paged_decode_attention(s["q"], st.k_cache, st.v_cache, s["block_tables"], s["context_lens"],
+                                       out=out, workspace=ws)
+        else:
+            ops.store_kvcache_and_decode_attention(s["q"], s["key"], s["value"], st.k_cache, st.v_cache,
+                                                   s["slot_mapping"], s["block_tables"], s["context_lens"],
+                                                   out=out, workspace=ws)
 
-    def decode(i):
-        s = st.steps[i % nsteps]
-        ops.paged_decode_attention(s["q"], st.k_cache, st.v_cache, s["block_tables"], s["context_lens"], out=out,
-                                   workspace=ws)
+    def step(i):
+        if mixed or args.separate_store:
+            s = st.steps[i % nsteps]
+            ops.store_kvcache(s["key"], s["value"], st.k_cache, st.v_cache, s["slot_mapping"])
+        attend(i)
+
+    launches_per_step = (5 if mixed else (3 if args.separate_store else 2))
 
     def barrier():
         if world > 1:
@@ -315,11 +362,10 @@ def npv_arm(args, rank, world, local_rank):
 
     bytes_steps = [step_bytes(wl, i % nsteps) for i in range(args.steps)]
     store_bytes = sum(b[0] for b in bytes_steps)
-    decode_bytes = sum(b[1] for b in bytes_steps)
+    attn_bytes = sum(b[1] for b in bytes_steps)
 
     for i in range(args.warmup):
-        store(i)
-        decode(i)
+        step(i)
     ops.check_device_errors()
 
     sampler = ClockSampler(local_rank) if rank == 0 else None
@@ -327,105 +373,176 @@ def npv_arm(args, rank, world, local_rank):
         sampler.start()
         time.sleep(0.3)
 
-    # ---- timed region 1: the plain step loop -> value
-    barrier()
-    torch.cuda.synchronize(dev)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(args.steps):
-        store(i)
-        decode(i)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    ms = max_over_ranks(e0.elapsed_time(e1))
+    def timed(fn, n):
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(n):
+            fn(i)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1))
 
-    # ---- timed region 2: the same loop with events around each decode call -> kernel roofline
+    # ---- timed region 1: the step loop -> value
+    ms = timed(step, args.steps)
+
+    # ---- timed region 2: events around each attention call -> kernel roofline
     barrier()
     torch.cuda.synchronize(dev)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for i in range(args.steps):
-        store(i)
+        if mixed or args.separate_store:
+            s = st.steps[i % nsteps]
+            ops.store_kvcache(s["key"], s["value"], st.k_cache, st.v_cache, s["slot_mapping"])
         evs[i][0].record(stream)
-        decode(i)
+        attend(i)
         evs[i][1].record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    dec_ms = [a.elapsed_time(b) for a, b in evs]
-    dec_mean = max_over_ranks(sum(dec_ms) / len(dec_ms))
+    call_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / args.steps)
+
+    extra = {}
+    if mixed:
+        extra = mixed_subbatches(args, wl, st, dev, stream, ops, W, timed)
 
     # keep the GPU loaded long enough for the clock sampler to see it
     t_end = time.time() + 1.5
     i = 0
     while time.time() < t_end:
-        for _ in range(50):
-            store(i)
-            decode(i)
+        for _ in range(20):
+            step(i)
             i += 1
         torch.cuda.synchronize(dev)
     clocks = sampler.stop() if sampler else None
     ops.check_device_errors()
 
-    # ---- end to end through the public API, host buffers, copies timed
     e2e = None
     if not args.no_e2e:
-        e2e = npv_e2e(args, wl, st, ws, dev, stream, ops, W, barrier, max_over_ranks)
+        e2e = npv_e2e(args, wl, st, ws, dev, stream, ops, W, barrier, max_over_ranks, step_fn_kind(args, mixed))
 
     peak, peak_kind = measured_peaks()
-    total_bytes = (store_bytes + decode_bytes) * world
+    total_bytes = (store_bytes + attn_bytes) * world
     value = total_bytes / (ms * 1e-3) / 1e9
-    achieved = (decode_bytes / args.steps) / (dec_mean * 1e-3) / 1e9
-    traffic = profiled_traffic(args.workload)
+    call_bytes = attn_bytes / args.steps + (0 if (mixed or args.separate_store) else store_bytes / args.steps)
+    achieved = call_bytes / (call_ms * 1e-3) / 1e9
     line = {
-        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "metric": METRIC if not mixed else MIXED_METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(wl),
-        "tokens_per_s": world * args.steps * wl.B / (ms * 1e-3),
+        "tokens_per_s": world * args.steps * wl.total_q / (ms * 1e-3),
         "pct_of_peak_hbm": 100.0 * value / world / peak,
-        "roofline": {"kernel": "npv_paged_decode_attention (split-KV kernel + merge kernel)", "bound": "hbm",
-                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                     else "fallback 6650 GB/s", "traffic": traffic,
-                     "algorithmic_bytes_per_launch": decode_bytes / args.steps,
-                     "mean_launch_ms": dec_mean},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
+    if not mixed:
+        line["roofline"] = {
+            "kernel": ("npv_paged_decode_attention" if args.separate_store else
+                       "npv_store_kvcache_and_decode_attention") + " (split-KV kernel + merge kernel)",
+            "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "peak_source": f"{peak_kind}: MEASURED_PEAKS.json hbm_gbs" if peak_kind == "measured"
+            else "fallback 6650 GB/s",
+            "traffic": profiled_traffic(args.workload) if not args.separate_store else None,
+            "algorithmic_bytes_per_launch": call_bytes, "mean_launch_ms": call_ms}
+    else:
+        line["roofline"] = extra.pop("roofline")
+        line.update(extra)
     if e2e is not None:
         line["e2e"] = e2e
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and not args.no_cpu_baseline and not mixed:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
 
 
-def npv_e2e(args, wl, st, ws, dev, stream, ops, W, barrier, max_over_ranks):
+def step_fn_kind(args, mixed):
+    return "mixed" if mixed else ("separate" if args.separate_store else "fused")
+
+
+def mixed_subbatches(args, wl, st, dev, stream, ops, W, timed):
+    """Time the prefill-only and decode-only parts of the mixed batch as their own calls."""
+    import torch
+
+    tflops_peak, tf_kind = measured_tflops()
+    hbm_peak, _ = measured_peaks()
+    s = st.steps[0]
+    cu = wl.cu_seqlens_q()
+    res = {}
+    for kind in ("prefill", "decode"):
+        seqs = [b for b in range(wl.B) if (wl.query_lens[b] > 1) == (kind == "prefill")]
+        rows = np.concatenate([np.arange(cu[b], cu[b + 1]) for b in seqs])
+        ridx = torch.from_numpy(rows).to(dev)
+        bidx = torch.from_numpy(np.array(seqs)).to(dev)
+        q = s["q"].index_select(0, ridx).contiguous()
+        bt = s["block_tables"].index_select(0, bidx).contiguous()
+        cl = s["context_lens"].index_select(0, bidx).contiguous()
+        cus = np.zeros(len(seqs) + 1, dtype=np.int32)
+        cus[1:] = np.cumsum(wl.query_lens[seqs])
+        cut = torch.from_numpy(cus).to(dev)
+        o = torch.empty_like(q)
+        wsz = ops.prefill_workspace_size(len(seqs), int(cus[-1]), wl.Hq, wl.Hkv, wl.D)
+        w = ops.alloc_workspace(wsz, dev)
+        mq = int(wl.query_lens[seqs].max())
+
+        def call(i, q=q, cut=cut, mq=mq, bt=bt, cl=cl, o=o, w=w):
+            ops.paged_prefill_attention(q, st.k_cache, st.v_cache, cut, mq, bt, cl, out=o, workspace=w)
+
+        for i in range(3):
+            call(i)
+        ms = timed(call, args.steps) / args.steps
+        _, nbytes = step_bytes(wl, 0, seqs)
+        fl = prefill_flops(wl, 0, seqs)
+        res[kind] = {"ms": ms, "gb_s": nbytes / (ms * 1e-3) / 1e9, "tflop_s": fl / (ms * 1e-3) / 1e12,
+                     "rows": int(cus[-1]), "seqs": len(seqs)}
+    pre = res["prefill"]
+    roof = {"kernel": "npv_paged_prefill_attention on the 16 prefill sequences (plan + tcgen05 kernel)",
+            "bound": "tensor", "achieved": pre["tflop_s"], "peak": tflops_peak, "unit": "TFLOP/s",
+            "frac": pre["tflop_s"] / tflops_peak, "peak_source": tf_kind, "traffic": None,
+            "algorithmic_flops_per_launch": prefill_flops(wl, 0, [b for b in range(wl.B) if wl.query_lens[b] > 1]),
+            "mean_launch_ms": pre["ms"]}
+    return {"roofline": roof, "prefill_part": pre,
+            "decode_part": dict(res["decode"], pct_of_peak_hbm=100 * res["decode"]["gb_s"] / hbm_peak)}
+
+
+def npv_e2e(args, wl, st, ws, dev, stream, ops, W, barrier, max_over_ranks, kind):
     """Host-resident inputs: each step copies its inputs H2D from pinned memory,
-    runs store + decode through the public API, and copies the output D2H."""
+    runs the step through the public API, and copies the output D2H."""
     import torch
 
     nsteps = wl.spec.num_steps
-    keys = ["q", "key", "value", "slot_mapping", "block_tables", "context_lens"]
+    keys = ["q", "key", "value", "slot_mapping", "block_tables", "context_lens", "cu_seqlens_q"]
     host = []
     for i in range(nsteps):
         s = st.steps[i]
         host.append({k: s[k].cpu().pin_memory() for k in keys})
     dbuf = {k: torch.empty_like(st.steps[0][k]) for k in keys}
-    out_dev = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device=dev)
-    out_host = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16).pin_memory()
-    h2d = sum(host[0][k].numel() * host[0][k].element_size() for k in keys)
+    out_dev = torch.empty((wl.total_q, wl.Hq, wl.D), dtype=torch.bfloat16, device=dev)
+    out_host = torch.empty((wl.total_q, wl.Hq, wl.D), dtype=torch.bfloat16).pin_memory()
+    used = keys if kind == "mixed" else keys[:-1]
+    h2d = sum(host[0][k].numel() * host[0][k].element_size() for k in used)
     d2h = out_host.numel() * out_host.element_size()
+    mq = st.steps[0]["max_seqlen_q"]
 
     def step(i):
         h = host[i % nsteps]
-        for k in keys:
+        for k in used:
             dbuf[k].copy_(h[k], non_blocking=True)
-        ops.store_kvcache(dbuf["key"], dbuf["value"], st.k_cache, st.v_cache, dbuf["slot_mapping"])
-        ops.paged_decode_attention(dbuf["q"], st.k_cache, st.v_cache, dbuf["block_tables"], dbuf["context_lens"],
-                                   out=out_dev, workspace=ws)
+        if kind == "fused":
+            ops.store_kvcache_and_decode_attention(dbuf["q"], dbuf["key"], dbuf["value"], st.k_cache, st.v_cache,
+                                                   dbuf["slot_mapping"], dbuf["block_tables"], dbuf["context_lens"],
+                                                   out=out_dev, workspace=ws)
+        else:
+            ops.store_kvcache(dbuf["key"], dbuf["value"], st.k_cache, st.v_cache, dbuf["slot_mapping"])
+            if kind == "mixed":
+                ops.paged_prefill_attention(dbuf["q"], st.k_cache, st.v_cache, dbuf["cu_seqlens_q"], mq,
+                                            dbuf["block_tables"], dbuf["context_lens"], out=out_dev, workspace=ws)
+            else:
+                ops.paged_decode_attention(dbuf["q"], st.k_cache, st.v_cache, dbuf["block_tables"],
+                                           dbuf["context_lens"], out=out_dev, workspace=ws)
         out_host.copy_(out_dev, non_blocking=True)
 
     for i in range(args.warmup):
@@ -445,7 +562,7 @@ def npv_e2e(args, wl, st, ws, dev, stream, ops, W, barrier, max_over_ranks):
     world = 1 if not torch.distributed.is_initialized() else torch.distributed.get_world_size()
     return {"value": world * nbytes / (ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms / args.steps,
-            "tokens_per_s": world * args.steps * wl.B / (ms * 1e-3)}
+            "tokens_per_s": world * args.steps * wl.total_q / (ms * 1e-3)}
 
 
 def main(argv=None):

@@ -150,6 +150,30 @@ NPV_API npv_status npv_paged_decode_attention(void *out, const void *q, int64_t 
                                       void *workspace, size_t workspace_bytes, npv_stream_t stream);
 
 /*
+ * One decode step's two jobs in one launch set: store each sequence's new key
+ * and value rows, then decode attention over the caches that include them
+ * ("3.1 Project overview and the four-layer architecture", section 3, Layer 4:
+ * the attention layer writes the new K/V, then attends).  The result equals
+ * npv_store_kvcache(key, value, ..., slot_mapping, num_tokens = num_seqs)
+ * followed by npv_paged_decode_attention, bit for bit.
+ *
+ *   key, value    [num_seqs, num_kv_heads, head_dim] bf16: token b is sequence
+ *                 b's new token, at position context_lens[b] - 1.  Strides as
+ *                 for npv_store_kvcache.
+ *   slot_mapping  [num_seqs] int32 (device): token b's slot, which must be the
+ *                 slot that sequence b's block table gives position
+ *                 context_lens[b] - 1 (the CTA that reads that position stores
+ *                 the token first).  A negative slot stores nothing.
+ *   other arguments and the workspace as for npv_paged_decode_attention.
+ */
+NPV_API npv_status npv_store_kvcache_and_decode_attention(
+    void *out, const void *q, int64_t q_seq_stride, const void *key, const void *value, int64_t key_token_stride,
+    int64_t value_token_stride, const int32_t *slot_mapping, void *k_cache, void *v_cache,
+    const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks, int32_t block_size, float scale,
+    void *workspace, size_t workspace_bytes, npv_stream_t stream);
+
+/*
  * Bytes of device workspace npv_paged_prefill_attention needs on the current
  * device.  Returns 0 for arguments the call would reject.
  */

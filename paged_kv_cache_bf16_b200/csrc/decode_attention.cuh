@@ -41,7 +41,7 @@ constexpr int kMaxStages = 8;
 constexpr int kStageBudgetBytes = 192 * 1024;
 constexpr int kHeaderBytes = 1024;
 
-enum : int32_t { kFlagFirst = 1, kFlagLast = 2, kFlagSkip = 4 };
+enum : int32_t { kFlagFirst = 1, kFlagLast = 2, kFlagSkip = 4, kFlagNewToken = 8 };
 
 struct StageInfo {
     int32_t unit;     // (sequence, head group) index
@@ -70,8 +70,14 @@ struct Params {
     int32_t num_head_groups;  // Hkv / HC
     int32_t num_stages;
     float scale_log2;  // softmax scale * log2(e)
+    // fused store (decode only): token b's key/value rows go to slot slot_mapping[b]
+    // before its sequence's last chunk is read; null when the call stores nothing
+    const uint16_t *key;
+    const uint16_t *value;
+    int64_t key_stride;    // elements between tokens
+    int64_t value_stride;
+    const int32_t *slot_mapping;
     // workspace
-    long long *meta;  // [grid][4]: total chunks, first unit, its first chunk, its end chunk
     float2 *part_ml;  // [grid][2][HC*g]: (running max, sum) of a partial unit
     float *part_o;    // [grid][2][HC*g][D]: unnormalised output of a partial unit
 };
@@ -117,6 +123,71 @@ __device__ __forceinline__ long long block_exclusive_scan(long long v, long long
     return scratch[warp] + incl - v;
 }
 
+// The contiguous range [c0, c1) of the flattened chunk list that CTA blockIdx.x of a
+// gridDim.x-CTA grid owns, and the unit holding chunk c0 with its chunk range
+// [s_first, e_first).  Every thread of the block must call this.
+struct Schedule {
+    long long total, c0, c1, u_first, s_first, e_first;
+};
+
+__device__ __forceinline__ Schedule compute_schedule(const Params &p, long long *sched, long long *scratch) {
+    const int NHG = p.num_head_groups;
+    const long long U = (long long)p.num_seqs * NHG;
+    const long long per = (U + blockDim.x - 1) / blockDim.x;
+    const long long lo = min(U, (long long)threadIdx.x * per);
+    const long long hi = min(U, lo + per);
+    long long mine = 0;
+    for (long long u = lo; u < hi; ++u) mine += seq_chunks(p, (int32_t)(u / NHG));
+    Schedule sc;
+    const long long excl = block_exclusive_scan(mine, scratch, &sc.total);
+    sc.c0 = (long long)blockIdx.x * sc.total / gridDim.x;
+    sc.c1 = (long long)(blockIdx.x + 1) * sc.total / gridDim.x;
+    if (sc.c0 < sc.c1 && mine > 0 && excl <= sc.c0 && sc.c0 < excl + mine) {
+        long long acc = excl;
+        for (long long u = lo; u < hi; ++u) {
+            const long long n = seq_chunks(p, (int32_t)(u / NHG));
+            if (sc.c0 < acc + n) {
+                sched[0] = u;
+                sched[1] = acc;
+                sched[2] = acc + n;
+                break;
+            }
+            acc += n;
+        }
+    }
+    __syncthreads();
+    if (sc.c0 < sc.c1) {
+        sc.u_first = sched[0];
+        sc.s_first = sched[1];
+        sc.e_first = sched[2];
+    } else {
+        sc.u_first = -1;
+        sc.s_first = sc.e_first = 0;
+    }
+    return sc;
+}
+
+// Fused store of token b's key/value rows for KV heads [h0, h0 + nh) into slot
+// slot_mapping[b] (a negative slot stores nothing), by the threads `lane` of `nthreads`.
+__device__ __forceinline__ void store_token_rows(const Params &p, int32_t b, int h0, int nh, int D, int lane,
+                                                 int nthreads) {
+    const int32_t slot = __ldg(p.slot_mapping + b);
+    if (slot < 0) return;
+    if ((long long)slot >= (long long)p.num_blocks * p.block_size) {
+        if (lane == 0) report_error(NPV_DEVERR_SLOT);
+        return;
+    }
+    const int64_t dst = ((int64_t)slot * p.num_kv_heads + h0) * D;
+    const uint16_t *ks = p.key + (int64_t)b * p.key_stride + (int64_t)h0 * D;
+    const uint16_t *vs = p.value + (int64_t)b * p.value_stride + (int64_t)h0 * D;
+    uint16_t *kc = const_cast<uint16_t *>(p.k_cache) + dst;
+    uint16_t *vc = const_cast<uint16_t *>(p.v_cache) + dst;
+    for (int v = lane; v < nh * D / 8; v += nthreads) {
+        st_global_v4(kc + v * 8, ld_nc_v4(ks + v * 8));
+        st_global_v4(vc + v * 8, ld_nc_v4(vs + v * 8));
+    }
+}
+
 template <int D, int G>
 struct Shape {
     static constexpr int LPR = D / 8;          // lanes per 16-byte-vector row
@@ -125,8 +196,12 @@ struct Shape {
     static constexpr int LOG_NI = NI == 8 ? 3 : (NI == 4 ? 2 : 1);
 };
 
+// Consumer warps (= KV heads) per CTA: 8, or 4 when g = 8 so that the larger
+// per-thread state (8 query heads) fits in registers.
+__host__ __device__ constexpr int max_heads_per_cta(int g) { return g >= 8 ? 4 : kMaxConsumerWarps; }
+
 template <int D, int G>
-__global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1) decode_split_kernel(const Params p) {
+__global__ void __launch_bounds__((max_heads_per_cta(G) + 1) * 32, 1) decode_split_kernel(const Params p) {
     using S = Shape<D, G>;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem);
@@ -156,40 +231,14 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1) decode_split_
 
     // ---- schedule: which contiguous range of the flattened chunk list is ours
     const int NHG = p.num_head_groups;
-    const long long U = (long long)p.num_seqs * NHG;
-    const long long per = (U + blockDim.x - 1) / blockDim.x;
-    const long long lo = min(U, (long long)threadIdx.x * per);
-    const long long hi = min(U, lo + per);
-    long long mine = 0;
-    for (long long u = lo; u < hi; ++u) mine += seq_chunks(p, (int32_t)(u / NHG));
-    long long total;
-    const long long excl = block_exclusive_scan(mine, scan_scratch, &total);
-    const long long c0 = (long long)blockIdx.x * total / gridDim.x;
-    const long long c1 = (long long)(blockIdx.x + 1) * total / gridDim.x;
-    if (c0 < c1 && mine > 0 && excl <= c0 && c0 < excl + mine) {
-        long long acc = excl;
-        for (long long u = lo; u < hi; ++u) {
-            const long long n = seq_chunks(p, (int32_t)(u / NHG));
-            if (c0 < acc + n) {
-                sched[0] = u;
-                sched[1] = acc;
-                sched[2] = acc + n;
-                break;
-            }
-            acc += n;
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        long long *m = p.meta + 4 * (size_t)blockIdx.x;
-        m[0] = total;
-        m[1] = c0 < c1 ? sched[0] : -1;
-        m[2] = c0 < c1 ? sched[1] : 0;
-        m[3] = c0 < c1 ? sched[2] : 0;
-    }
-    if (c0 >= c1) return;
-    const long long u_first = sched[0];
-    const long long s_first = sched[1];
+    const Schedule sc = compute_schedule(p, sched, scan_scratch);
+    // the merge kernel may now be scheduled; it waits for this grid before
+    // reading any partial
+    grid_launch_dependents();
+    if (sc.c0 >= sc.c1) return;
+    const long long c0 = sc.c0, c1 = sc.c1;
+    const long long u_first = sc.u_first;
+    const long long s_first = sc.s_first;
 
     if (warp == HC) {
         // ===================== producer warp =====================
@@ -236,6 +285,9 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1) decode_split_
                 }
                 if (lane == 0) {
                     int32_t flags = (i == 0 ? kFlagFirst : 0) | (i == seg_len - 1 ? kFlagLast : 0);
+                    // a fused store: this segment ends with the unit's last chunk, which
+                    // holds the new token (the consumers store and substitute it)
+                    if (i == 0 && p.key != nullptr && k + seg_len == nC) flags |= kFlagNewToken;
                     if (!valid) {
                         flags |= kFlagSkip;
                         report_error(NPV_DEVERR_BLOCK_ID);
@@ -300,6 +352,9 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1) decode_split_
 
     float qf[G][8], o[G][8], m_run[G], l_run[G];
     int32_t b = 0, hg = 0;
+    // fused store: this lane's 8-element slices of the new token's K and V rows
+    uint4 new_k = make_uint4(0, 0, 0, 0), new_v = make_uint4(0, 0, 0, 0);
+    int32_t new_slot = -1;
     int stage = 0;
     uint32_t fparity = 0;
     const long long nchunks = c1 - c0;
@@ -323,6 +378,39 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1) decode_split_
                 m_run[j] = -INFINITY;
                 l_run[j] = 0.f;
             }
+            new_slot = -1;
+            if (inf.flags & kFlagNewToken) {
+                // fetch now; used when the segment's last chunk arrives
+                const int32_t slot = __ldg(p.slot_mapping + b);
+                if (slot >= 0 && (long long)slot < (long long)p.num_blocks * p.block_size) {
+                    new_slot = slot;
+                    const int64_t h = (int64_t)(hg * HC + warp) * D + sub * 8;
+                    new_k = ld_nc_v4(p.key + (int64_t)b * p.key_stride + h);
+                    new_v = ld_nc_v4(p.value + (int64_t)b * p.value_stride + h);
+                } else if (slot >= 0 && lane == 0) {
+                    report_error(NPV_DEVERR_SLOT);
+                }
+            }
+        }
+        if ((inf.flags & kFlagLast) && new_slot >= 0) {
+            // the unit's last chunk: put the new token into the stage (its cache
+            // slot may not hold it yet) and into the cache
+            const int tl = inf.n_valid - 1;
+            if (rg == 0) {
+                const uint32_t off = (uint32_t)(((tl * HC + warp) * D + sub * 8) * 2);
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_addr(stage_k) + stage * stage_bytes +
+                                                                            off),
+                             "r"(new_k.x), "r"(new_k.y), "r"(new_k.z), "r"(new_k.w)
+                             : "memory");
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_addr(stage_v) + stage * stage_bytes +
+                                                                            off),
+                             "r"(new_v.x), "r"(new_v.y), "r"(new_v.z), "r"(new_v.w)
+                             : "memory");
+                const int64_t dst = ((int64_t)new_slot * p.num_kv_heads + hg * HC + warp) * D + sub * 8;
+                st_global_v4(const_cast<uint16_t *>(p.k_cache) + dst, new_k);
+                st_global_v4(const_cast<uint16_t *>(p.v_cache) + dst, new_v);
+            }
+            __syncwarp();
         }
         if (!(inf.flags & kFlagSkip)) {
             const bool full = inf.n_valid == kChunk;
@@ -473,21 +561,27 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1) decode_split_
 }
 
 // Finish what the split kernel left: combine the partials of every unit that
-// was cut by a CTA boundary (each merge CTA takes the unit that ends inside its
-// split CTA's range), and write zero rows (reporting invalid lengths) for
-// sequences the split kernel had no chunks for.
+// was cut by a CTA boundary (merge CTA c takes the unit that starts before
+// split CTA c's range and ends inside it), and write zero rows (reporting
+// invalid lengths) for sequences the split kernel had no chunks for.  The grid
+// has the split kernel's size.  Everything that does not read the split
+// kernel's output runs before griddepcontrol.wait, overlapping the split
+// kernel's tail; every CTA waits before it exits.
 __global__ void __launch_bounds__(256) decode_merge_kernel(const Params p, int head_dim) {
-    grid_dependency_wait();
+    __shared__ long long sched[4];
+    __shared__ long long scratch[16];
     const int D = head_dim;
-    const int c = blockIdx.x;
+    const long long c = blockIdx.x;
     const long long G = gridDim.x;
     const int HC = p.heads_per_cta;
     const int g = p.num_q_heads / p.num_kv_heads;
     const int HCG = HC * g;
     const int NHG = p.num_head_groups;
 
+    const Schedule sc = compute_schedule(p, sched, scratch);
+
     // (1) rows with no chunks on this path
-    for (long long b = c + (long long)G * threadIdx.x; b < p.num_seqs; b += G * blockDim.x) {
+    for (long long b = c + G * threadIdx.x; b < p.num_seqs; b += G * blockDim.x) {
         const int32_t L = __ldg(p.context_lens + b);
         if (p.cu_seqlens_q != nullptr) {
             const int32_t cb = __ldg(p.cu_seqlens_q + b), ce = __ldg(p.cu_seqlens_q + b + 1);
@@ -501,16 +595,18 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const Params p, int h
         if (L <= 0 || bad) {
             uint4 *orow = reinterpret_cast<uint4 *>(p.out + query_row(p, (int32_t)b) * (int64_t)p.num_q_heads * D);
             for (int i = 0; i < p.num_q_heads * D / 8; ++i) orow[i] = make_uint4(0, 0, 0, 0);
+            // a fused store still writes this sequence's token
+            if (p.key != nullptr) store_token_rows(p, (int32_t)b, 0, p.num_kv_heads, D, 0, 1);
         }
     }
 
     // (2) the unit that starts before this CTA's range and ends inside it
-    const long long *m = p.meta + 4 * (size_t)c;
-    const long long N = m[0], u = m[1], S = m[2], E = m[3];
-    const long long c0 = (long long)c * N / G, c1 = (long long)(c + 1) * N / G;
-    if (c0 >= c1 || u < 0 || !(S < c0 && E <= c1)) return;
-    const long long ca = ((S + 1) * G - 1) / N;  // split CTA holding the unit's first chunk
-    const int sa = (S == ca * N / G) ? 0 : 1;
+    const bool work = sc.c0 < sc.c1 && sc.s_first < sc.c0 && sc.e_first <= sc.c1;
+    const long long N = sc.total, u = sc.u_first, S = sc.s_first;
+    const long long ca = work ? ((S + 1) * G - 1) / N : 0;  // split CTA holding the unit's first chunk
+    const int sa = (work && S == ca * N / G) ? 0 : 1;
+    grid_dependency_wait();
+    if (!work) return;
     const int32_t b = (int32_t)(u / NHG), hg = (int32_t)(u % NHG);
     uint16_t *orow = p.out + query_row(p, b) * (int64_t)p.num_q_heads * D + (int64_t)hg * HCG * D;
     for (int idx = threadIdx.x; idx < HCG * D / 4; idx += blockDim.x) {

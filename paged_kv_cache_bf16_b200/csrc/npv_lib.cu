@@ -79,14 +79,14 @@ struct DecodeConfig {
     int stages = 0;
     int grid = 0;
     size_t smem = 0;
-    size_t ws_meta = 0, ws_ml = 0, ws_o = 0, ws_total = 0;
+    size_t ws_ml = 0, ws_o = 0, ws_total = 0;
 };
 
 bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
 
-// Largest divisor of Hkv that is at most 8 (one consumer warp per KV head).
-int pick_heads_per_cta(int num_kv_heads) {
-    for (int hc = 8; hc >= 1; --hc)
+// Largest divisor of Hkv within the kernel's consumer-warp budget (one warp per KV head).
+int pick_heads_per_cta(int num_kv_heads, int g) {
+    for (int hc = npv::decode::max_heads_per_cta(g); hc >= 1; --hc)
         if (num_kv_heads % hc == 0) return hc;
     return 1;
 }
@@ -99,7 +99,7 @@ npv_status decode_config(int num_q_heads, int num_kv_heads, int head_dim, Decode
     const DeviceInfo *dev = current_device();
     if (!dev) return NPV_ERR_CUDA;
     cfg->group = g;
-    cfg->heads_per_cta = pick_heads_per_cta(num_kv_heads);
+    cfg->heads_per_cta = pick_heads_per_cta(num_kv_heads, g);
     cfg->head_groups = num_kv_heads / cfg->heads_per_cta;
     const int hc = cfg->heads_per_cta;
     const size_t stage_bytes = 2ull * npv::decode::kChunk * hc * head_dim * 2;
@@ -112,10 +112,9 @@ npv_status decode_config(int num_q_heads, int num_kv_heads, int head_dim, Decode
     if ((int)cfg->smem > dev->max_smem_optin) return NPV_ERR_UNSUPPORTED;
     cfg->grid = dev->sm_count;
     const size_t hcg = (size_t)hc * g;
-    cfg->ws_meta = align_up((size_t)cfg->grid * 4 * sizeof(long long), 256);
     cfg->ws_ml = align_up((size_t)cfg->grid * 2 * hcg * sizeof(float2), 256);
     cfg->ws_o = align_up((size_t)cfg->grid * 2 * hcg * head_dim * sizeof(float), 256);
-    cfg->ws_total = cfg->ws_meta + cfg->ws_ml + cfg->ws_o;
+    cfg->ws_total = cfg->ws_ml + cfg->ws_o;
     return NPV_OK;
 }
 
@@ -149,13 +148,22 @@ cudaError_t dispatch_decode_split(int D, const npv::decode::Params &p, const Dec
     return cudaErrorInvalidValue;
 }
 
-// Shared by the decode call and the decode rows of the prefill call.
+// New K/V rows stored by a fused store + decode call (one token per sequence).
+struct FusedStore {
+    const void *key;
+    const void *value;
+    int64_t key_stride;
+    int64_t value_stride;
+    const int32_t *slot_mapping;
+};
+
+// Shared by the decode calls and the decode rows of the prefill call.
 npv_status run_decode(void *out, const void *q, int64_t q_row_stride, const int32_t *cu_seqlens_q, int32_t total_q,
                       const void *k_cache, const void *v_cache, const int32_t *block_tables,
                       int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs,
                       int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks,
                       int32_t block_size, float scale, void *workspace, const DecodeConfig &cfg,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, const FusedStore *store = nullptr) {
     npv::decode::Params p = {};
     p.out = static_cast<uint16_t *>(out);
     p.q = static_cast<const uint16_t *>(q);
@@ -178,9 +186,15 @@ npv_status run_decode(void *out, const void *q, int64_t q_row_stride, const int3
     const float s = scale > 0.f ? scale : (float)(1.0 / std::sqrt((double)head_dim));
     p.scale_log2 = s * 1.4426950408889634f;
     char *ws = static_cast<char *>(workspace);
-    p.meta = reinterpret_cast<long long *>(ws);
-    p.part_ml = reinterpret_cast<float2 *>(ws + cfg.ws_meta);
-    p.part_o = reinterpret_cast<float *>(ws + cfg.ws_meta + cfg.ws_ml);
+    p.part_ml = reinterpret_cast<float2 *>(ws);
+    p.part_o = reinterpret_cast<float *>(ws + cfg.ws_ml);
+    if (store) {
+        p.key = static_cast<const uint16_t *>(store->key);
+        p.value = static_cast<const uint16_t *>(store->value);
+        p.key_stride = store->key_stride;
+        p.value_stride = store->value_stride;
+        p.slot_mapping = store->slot_mapping;
+    }
     cudaError_t e = dispatch_decode_split(head_dim, p, cfg, stream);
     if (e != cudaSuccess) return NPV_ERR_CUDA;
     e = launch_pdl(npv::decode::decode_merge_kernel, dim3(cfg.grid), dim3(256), 0, stream, p, (int)head_dim);
@@ -375,6 +389,43 @@ npv_status npv_paged_decode_attention(void *out, const void *q, int64_t q_seq_st
     return run_decode(out, q, q_seq_stride, nullptr, num_seqs, k_cache, v_cache, block_tables, max_blocks_per_seq,
                       context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, scale,
                       workspace, cfg, (cudaStream_t)stream);
+}
+
+npv_status npv_store_kvcache_and_decode_attention(
+    void *out, const void *q, int64_t q_seq_stride, const void *key, const void *value, int64_t key_token_stride,
+    int64_t value_token_stride, const int32_t *slot_mapping, void *k_cache, void *v_cache,
+    const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks, int32_t block_size, float scale,
+    void *workspace, size_t workspace_bytes, npv_stream_t stream) {
+    if (num_seqs < 0 || max_blocks_per_seq <= 0 || !cache_shape_ok(num_blocks, block_size, num_kv_heads, head_dim))
+        return NPV_ERR_INVALID_ARG;
+    if (num_q_heads <= 0 || num_q_heads % num_kv_heads != 0) return NPV_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return NPV_ERR_INVALID_ARG;
+    if (block_size % 16 != 0) return NPV_ERR_UNSUPPORTED;
+    DecodeConfig cfg;
+    npv_status st = decode_config(num_q_heads, num_kv_heads, head_dim, &cfg);
+    if (st != NPV_OK) return st;
+    if (num_seqs == 0) return NPV_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !key || !value || !slot_mapping)
+        return NPV_ERR_INVALID_ARG;
+    const int64_t qrow = (int64_t)num_q_heads * head_dim;
+    const int64_t kvrow = (int64_t)num_kv_heads * head_dim;
+    if (q_seq_stride == 0) q_seq_stride = qrow;
+    if (key_token_stride == 0) key_token_stride = kvrow;
+    if (value_token_stride == 0) value_token_stride = kvrow;
+    if (q_seq_stride < qrow || (q_seq_stride * 2) % 16 != 0) return NPV_ERR_INVALID_ARG;
+    if (key_token_stride < kvrow || value_token_stride < kvrow || (key_token_stride * 2) % 16 != 0 ||
+        (value_token_stride * 2) % 16 != 0)
+        return NPV_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(key) ||
+        !aligned16(value))
+        return NPV_ERR_INVALID_ARG;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < cfg.ws_total)
+        return NPV_ERR_WORKSPACE;
+    const FusedStore fs = {key, value, key_token_stride, value_token_stride, slot_mapping};
+    return run_decode(out, q, q_seq_stride, nullptr, num_seqs, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                      context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, scale,
+                      workspace, cfg, (cudaStream_t)stream, &fs);
 }
 
 size_t npv_paged_prefill_workspace_size(int32_t num_seqs, int32_t total_q, int32_t num_q_heads,

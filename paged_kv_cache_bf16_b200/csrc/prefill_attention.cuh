@@ -13,14 +13,19 @@
 //   * Work item = (sequence, KV head, tile of 128 MMA rows).  The 128 rows pack
 //     128/g positions x the g query heads of one GQA group, so every K/V tile
 //     loaded from HBM feeds all g heads (row r = position * g + head).
-//   * A one-CTA plan kernel lists the (sequence, row-tile) pairs, counting-sorted
-//     by their number of 128-key KV tiles, longest first.  The persistent main
-//     kernel (one CTA per SM) takes items from that list in snake order.
-//   * Warp roles: warp 4 issues TMA loads (Q once per item, K and V tiles of 128
-//     keys through a 2-stage ring; block ids come from the block table a
-//     32-entry window at a time, one TMA box per block piece); warp 5 owns tensor
-//     memory and issues tcgen05.mma from one thread; warps 0-3 run the softmax,
-//     one TMEM lane (= one query row) per thread.
+//   * A one-CTA plan kernel lists the (sequence, row-tile) pairs: sequences
+//     counting-sorted by KV length, longest first, each sequence's tiles
+//     contiguous (so the items that read the same K/V run at the same time and
+//     share it through L2).  The persistent main kernel (one CTA per SM) takes
+//     items (pair, KV head) from that list in snake order.
+//   * Warp roles: warp 4 issues the TMA loads of Q (once per item) and of the
+//     K tiles (128 keys) through a 3-stage ring, warp 6 those of the V tiles
+//     through a 2-stage ring; block ids come from the block table a 32-entry
+//     window at a time, one TMA box per block piece.  A K stage is released as
+//     soon as its S = Q K^T product completes, so K loads run ahead of the P.V
+//     products.  Warp 5 owns tensor memory and issues tcgen05.mma from one
+//     thread; warps 0-3 run the softmax, one TMEM lane (= one query row) per
+//     thread.
 //   * Tensor memory holds S twice (so S for tile j+1 is computed while the
 //     softmax reads tile j) and the O accumulator.  S = Q K^T reads Q and K as
 //     K-major 128-byte-swizzled operands; O += P V reads P (bf16, written by the
@@ -40,10 +45,12 @@ namespace prefill {
 
 constexpr int kTileM = 128;   // query rows per item (MMA M)
 constexpr int kTileN = 128;   // keys per KV tile (MMA N of S, K of P.V)
-constexpr int kStages = 2;    // K/V ring depth
-constexpr int kThreads = 192; // 4 softmax warps, producer, MMA
-constexpr int kProducerWarp = 4;
+constexpr int kKStages = 3;   // K ring depth (a K stage is free once S = Q K^T is done)
+constexpr int kVStages = 2;   // V ring depth (a V stage is free once O += P V is done)
+constexpr int kThreads = 224; // 4 softmax warps, K producer, MMA, V producer
+constexpr int kKProducerWarp = 4;
 constexpr int kMmaWarp = 5;
+constexpr int kVProducerWarp = 6;
 constexpr int kTmemCols = 512;
 constexpr int kBuckets = 4096;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -76,8 +83,8 @@ struct Smem {
     static constexpr int kP = kTileM * kTileN * 2;
     static constexpr int q = kHeader;
     static constexpr int k = q + kQ;
-    static constexpr int v = k + kStages * kKV;
-    static constexpr int p = v + kStages * kKV;
+    static constexpr int v = k + kKStages * kKV;
+    static constexpr int p = v + kVStages * kKV;
     static constexpr int total = p + kP;
 };
 
@@ -172,18 +179,16 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const Params p, int 
     long long base = decode::block_exclusive_scan(mine, scratch, &total);
     (void)base;
     __syncthreads();
-    // histogram of KV-tile counts (reversed so that the longest come first)
+    // Sequences are ordered by their KV length, longest first (counting sort on
+    // 128-key tiles); each sequence's row tiles stay contiguous, last tile first,
+    // so the CTAs reading the same K/V run together and share it through L2.
     for (int b = lo; b < hi; ++b) {
         int32_t n;
         bool bad;
         if (!prefill_seq(p, b, &n, &bad)) continue;
         const int32_t L = __ldg(p.context_lens + b);
-        for (int qt = 0; qt * ppt < n; ++qt) {
-            const int npos = min(ppt, n - qt * ppt);
-            const int kv_end = min(L, L - n + qt * ppt + npos);
-            const int nt = min(kBuckets - 1, (kv_end + kTileN - 1) / kTileN);
-            atomicAdd(&hist[kBuckets - 1 - nt], 1);
-        }
+        const int nt = min(kBuckets - 1, (L + kTileN - 1) / kTileN);
+        atomicAdd(&hist[kBuckets - 1 - nt], (n + ppt - 1) / ppt);
     }
     __syncthreads();
     // exclusive scan of the histogram: 4 buckets per thread
@@ -211,13 +216,11 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const Params p, int 
         bool bad;
         if (!prefill_seq(p, b, &n, &bad)) continue;
         const int32_t L = __ldg(p.context_lens + b);
-        for (int qt = 0; qt * ppt < n; ++qt) {
-            const int npos = min(ppt, n - qt * ppt);
-            const int kv_end = min(L, L - n + qt * ppt + npos);
-            const int nt = min(kBuckets - 1, (kv_end + kTileN - 1) / kTileN);
-            const int pos = atomicAdd(&hist[kBuckets - 1 - nt], 1);
-            if (pos < p.max_pairs) p.plan_pairs[pos] = make_int2(b, qt);
-        }
+        const int nt = min(kBuckets - 1, (L + kTileN - 1) / kTileN);
+        const int nqt = (n + ppt - 1) / ppt;
+        const int pos = atomicAdd(&hist[kBuckets - 1 - nt], nqt);
+        for (int k = 0; k < nqt; ++k)
+            if (pos + k < p.max_pairs) p.plan_pairs[pos + k] = make_int2(b, nqt - 1 - k);
     }
     if (tid == 0) p.plan_count[0] = (int32_t)min(total, (long long)p.max_pairs);
 }
@@ -225,6 +228,38 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const Params p, int 
 // ---------------------------------------------------------------------------
 // main kernel
 // ---------------------------------------------------------------------------
+
+// Block ids of the (up to 8) TMA boxes of KV tile t of an item: box i covers
+// keys t*128 + i*box_tokens; boxes past the item's keys or with an invalid
+// block id get -1.  Warp-collective (the block-table window lives in lanes).
+__device__ __forceinline__ int tile_boxes(const Params &p, const Item &it, const int32_t *bt_row, int t, int lane,
+                                          int &win, int &win_val, int (&blk_of_box)[8]) {
+    const int BS = p.block_size;
+    const int nbox = kTileN / p.box_tokens;
+    const int kv0 = t * kTileN;
+    int nload = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        blk_of_box[i] = -1;
+        if (i >= nbox) continue;
+        const int ks = kv0 + i * p.box_tokens;
+        if (ks >= it.kv_end) continue;  // warp-uniform
+        const int li = ks / BS;
+        if ((li >> 5) != win) {
+            win = li >> 5;
+            const int e = (win << 5) + lane;
+            win_val = e < p.max_blocks_per_seq ? __ldg(bt_row + e) : -1;
+        }
+        const int blk = __shfl_sync(0xffffffffu, win_val, li & 31);
+        if (blk >= 0 && blk < p.num_blocks) {
+            blk_of_box[i] = blk;
+            ++nload;
+        } else if (lane == 0) {
+            report_error(NPV_DEVERR_BLOCK_ID);
+        }
+    }
+    return nload;
+}
 
 #define NPV_WAIT(bar, parity)                     \
     do {                                          \
@@ -246,17 +281,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
     uint64_t *q_full = bars + 0;
     uint64_t *q_empty = bars + 1;
-    uint64_t *k_full = bars + 2;     // [2]
-    uint64_t *v_full = bars + 4;     // [2]
-    uint64_t *kv_empty = bars + 6;   // [2]
-    uint64_t *s_full = bars + 8;     // [2]
-    uint64_t *s_free = bars + 10;    // [2]
-    uint64_t *p_full = bars + 12;
-    uint64_t *p_empty = bars + 13;
-    uint64_t *o_full = bars + 14;
-    uint64_t *o_free = bars + 15;
-    uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(bars + 16);
-    int *abort_flag = reinterpret_cast<int *>(bars + 17);
+    uint64_t *k_full = bars + 2;     // [kKStages]
+    uint64_t *k_empty = bars + 5;    // [kKStages]
+    uint64_t *v_full = bars + 8;     // [kVStages]
+    uint64_t *v_empty = bars + 10;   // [kVStages]
+    uint64_t *s_full = bars + 12;    // [2]
+    uint64_t *s_free = bars + 14;    // [2]
+    uint64_t *p_full = bars + 16;
+    uint64_t *p_empty = bars + 17;
+    uint64_t *o_full = bars + 18;
+    uint64_t *o_free = bars + 19;
+    uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(bars + 20);
+    int *abort_flag = reinterpret_cast<int *>(bars + 21);
     uint8_t *sQ = smem + L::q;
     uint8_t *sK = smem + L::k;
     uint8_t *sV = smem + L::v;
@@ -269,10 +305,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
         mbar_init(q_empty, 1);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kKStages; ++s) {
             mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < kVStages; ++s) {
             mbar_init(&v_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+            mbar_init(&v_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
             mbar_init(&s_full[s], 1);
             mbar_init(&s_free[s], 4);
         }
@@ -283,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == kProducerWarp && lane == 0) {
+    if (warp == kKProducerWarp && lane == 0) {
         tc::prefetch_tensormap(&qmap);
         tc::prefetch_tensormap(&kmap);
         tc::prefetch_tensormap(&vmap);
@@ -301,8 +342,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const long long n_items = (long long)p.plan_count[0] * p.num_kv_heads;
     const long long rounds = (n_items + gridDim.x - 1) / gridDim.x;
 
-    if (warp == kProducerWarp) {
-        // ============================ TMA producer ============================
+    if (warp == kKProducerWarp || warp == kVProducerWarp) {
+        // ============================ TMA producers ============================
+        const bool is_k = warp == kKProducerWarp;
+        const int nstages = is_k ? kKStages : kVStages;
+        uint64_t *full = is_k ? k_full : v_full;
+        uint64_t *empty = is_k ? k_empty : v_empty;
+        uint8_t *ring = is_k ? sK : sV;
+        const CUtensorMap *map = is_k ? &kmap : &vmap;
         uint32_t q_iter = 0, kv_iter = 0;
         const int BS = p.block_size;
         for (long long r = 0; r < rounds; ++r) {
@@ -311,58 +358,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Item it = load_item<G>(p, idx);
             const int32_t *bt_row = p.block_tables + (size_t)it.b * p.max_blocks_per_seq;
             int win = -1, win_val = -1;
-            NPV_WAIT(q_empty, (q_iter & 1) ^ 1);
-            if (lane == 0) {
-                mbar_arrive_expect_tx(q_full, (uint32_t)L::kQ);
-                for (int db = 0; db < kDBlocks; ++db)
-                    tc::tma_load_3d(sQ + db * (kTileM * 128), &qmap, db * 64, it.h * G, it.row0 + it.p0, q_full);
-            }
-            ++q_iter;
-            for (int t = 0; t < it.ntiles; ++t, ++kv_iter) {
-                const int s = kv_iter & 1;
-                NPV_WAIT(&kv_empty[s], ((kv_iter >> 1) & 1) ^ 1);
-                const int kv0 = t * kTileN;
-                const int nbox = kTileN / p.box_tokens;
-                int blk_of_box[8];
-                int nload = 0;
-                for (int i = 0; i < nbox; ++i) {
-                    const int ks = kv0 + i * p.box_tokens;
-                    blk_of_box[i] = -1;
-                    if (ks >= it.kv_end) continue;  // warp-uniform
-                    const int li = ks / BS;
-                    if ((li >> 5) != win) {
-                        win = li >> 5;
-                        const int e = (win << 5) + lane;
-                        win_val = e < p.max_blocks_per_seq ? __ldg(bt_row + e) : -1;
-                    }
-                    const int blk = __shfl_sync(0xffffffffu, win_val, li & 31);
-                    if (blk >= 0 && blk < p.num_blocks) {
-                        blk_of_box[i] = blk;
-                        ++nload;
-                    } else if (lane == 0) {
-                        report_error(NPV_DEVERR_BLOCK_ID);
-                    }
+            if (is_k) {
+                NPV_WAIT(q_empty, (q_iter & 1) ^ 1);
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(q_full, (uint32_t)L::kQ);
+                    for (int db = 0; db < kDBlocks; ++db)
+                        tc::tma_load_3d(sQ + db * (kTileM * 128), &qmap, db * 64, it.h * G, it.row0 + it.p0,
+                                        q_full);
                 }
+                ++q_iter;
+            }
+            for (int t = 0; t < it.ntiles; ++t, ++kv_iter) {
+                const int s = (int)(kv_iter % nstages);
+                NPV_WAIT(&empty[s], ((kv_iter / nstages) & 1) ^ 1);
+                int blk_of_box[8];
+                const int nload = tile_boxes(p, it, bt_row, t, lane, win, win_val, blk_of_box);
                 if (lane == 0) {
                     const uint32_t bytes = (uint32_t)(nload * p.box_tokens * 128 * kDBlocks);
-                    uint8_t *dk = sK + s * L::kKV;
-                    uint8_t *dv = sV + s * L::kKV;
-                    if (bytes) {
-                        mbar_arrive_expect_tx(&k_full[s], bytes);
-                        mbar_arrive_expect_tx(&v_full[s], bytes);
-                    } else {
-                        mbar_arrive(&k_full[s]);
-                        mbar_arrive(&v_full[s]);
-                    }
-                    for (int i = 0; i < nbox; ++i) {
+                    uint8_t *dst = ring + s * L::kKV;
+                    if (bytes)
+                        mbar_arrive_expect_tx(&full[s], bytes);
+                    else
+                        mbar_arrive(&full[s]);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
                         if (blk_of_box[i] < 0) continue;
-                        const int ks = kv0 + i * p.box_tokens;
+                        const int ks = t * kTileN + i * p.box_tokens;
                         const int slot_row = blk_of_box[i] * BS + ks % BS;
-                        for (int db = 0; db < kDBlocks; ++db) {
-                            const int off = db * kBlockBytes + i * p.box_tokens * 128;
-                            tc::tma_load_3d(dk + off, &kmap, db * 64, it.h, slot_row, &k_full[s]);
-                            tc::tma_load_3d(dv + off, &vmap, db * 64, it.h, slot_row, &v_full[s]);
-                        }
+                        for (int db = 0; db < kDBlocks; ++db)
+                            tc::tma_load_3d(dst + db * kBlockBytes + i * p.box_tokens * 128, map, db * 64, it.h,
+                                            slot_row, &full[s]);
                     }
                 }
                 __syncwarp();
@@ -386,8 +411,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (t < it.ntiles) {
                     // ---- S[t % 2] = Q K_t^T
                     const uint32_t T = kv_iter + t;
-                    const int s = T & 1;
-                    NPV_WAIT(&k_full[s], (T >> 1) & 1);
+                    const int s = T & 1;              // S buffer
+                    const int ks = (int)(T % kKStages);  // K stage
+                    NPV_WAIT(&k_full[ks], (T / kKStages) & 1);
                     NPV_WAIT(&s_free[s], ((T >> 1) & 1) ^ 1);
                     tc::fence_after_sync();
                     if (lane == 0) {
@@ -395,10 +421,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int k = 0; k < D / 16; ++k) {
                             const uint32_t off = (k >> 2) * kBlockBytes + (k & 3) * 32;
                             tc::mma_bf16_ss(tmem + s * kTileN, tc::smem_desc_sw128(q_addr + off, 16, 1024),
-                                            tc::smem_desc_sw128(k_addr + s * L::kKV + off, 16, 1024), idesc_s,
+                                            tc::smem_desc_sw128(k_addr + ks * L::kKV + off, 16, 1024), idesc_s,
                                             k > 0);
                         }
                         tc::mma_commit(&s_full[s]);
+                        tc::mma_commit(&k_empty[ks]);
                         if (t == it.ntiles - 1) tc::mma_commit(q_empty);
                     }
                     __syncwarp();
@@ -407,9 +434,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // ---- O (+)= P_{t-1} V_{t-1}
                     const int tp = t - 1;
                     const uint32_t T = kv_iter + tp;
-                    const int s = T & 1;
+                    const int s = (int)(T % kVStages);  // V stage
                     NPV_WAIT(p_full, T & 1);
-                    NPV_WAIT(&v_full[s], (T >> 1) & 1);
+                    NPV_WAIT(&v_full[s], (T / kVStages) & 1);
                     if (tp == 0) NPV_WAIT(o_free, (item_iter & 1) ^ 1);
                     const int valid = min(kTileN, it.kv_end - tp * kTileN);
                     const int ksteps = (valid + 15) / 16;
@@ -436,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                             tc::smem_desc_sw128(v_addr + s * L::kKV + voff, kBlockBytes, 1024),
                                             idesc_o, tp > 0 || k > 0);
                         }
-                        tc::mma_commit(&kv_empty[s]);
+                        tc::mma_commit(&v_empty[s]);
                         tc::mma_commit(p_empty);
                         if (tp == it.ntiles - 1) tc::mma_commit(o_full);
                     }
@@ -467,14 +494,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::fence_after_sync();
                 float sv[kTileN];
                 {
-                    uint32_t raw[32];
+                    // all four TMEM loads in flight before a single wait
+                    uint32_t raw[kTileN / 32][32];
 #pragma unroll
-                    for (int c = 0; c < kTileN / 32; ++c) {
-                        tc::tmem_ld32(tmem + lane_off + sb * kTileN + c * 32, raw);
-                        tc::tmem_wait_ld();
+                    for (int c = 0; c < kTileN / 32; ++c) tc::tmem_ld32(tmem + lane_off + sb * kTileN + c * 32, raw[c]);
+                    tc::tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(raw[e]);
-                    }
+                    for (int c = 0; c < kTileN / 32; ++c)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(raw[c][e]);
                 }
                 tc::fence_before_sync();
                 __syncwarp();
@@ -485,9 +513,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int c = 0; c < kTileN; ++c)
                         if (kv0 + c > lim) sv[c] = -INFINITY;
                 }
-                float mx = sv[0];
+                // row max with 8 independent chains
+                float mx8[8];
 #pragma unroll
-                for (int c = 1; c < kTileN; ++c) mx = fmaxf(mx, sv[c]);
+                for (int e = 0; e < 8; ++e) mx8[e] = sv[e];
+#pragma unroll
+                for (int c = 8; c < kTileN; c += 8)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], sv[c + e]);
+                const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
                 const float m_tile = mx * p.scale_log2;
                 if (t == 0) {
                     m = m_tile;
@@ -499,15 +534,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                         NPV_WAIT(p_empty, (T - 1) & 1);
                         tc::fence_after_sync();
                         const float alpha = need ? fast_exp2(m - m_new) : 1.0f;
+                        // 32 columns at a time: the scores are still live in registers
 #pragma unroll
-                        for (int c = 0; c < D / 32; ++c) {
-                            uint32_t raw[32];
-                            const uint32_t ta = tmem + lane_off + 2 * kTileN + c * 32;
-                            tc::tmem_ld32(ta, raw);
+                        for (int c0 = 0; c0 < D / 32; c0 += 1) {
+                            uint32_t raw[1][32];
+#pragma unroll
+                            for (int c = 0; c < 1; ++c)
+                                tc::tmem_ld32(tmem + lane_off + 2 * kTileN + (c0 + c) * 32, raw[c]);
                             tc::tmem_wait_ld();
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
-                            tc::tmem_st32(ta, raw);
+                            for (int c = 0; c < 1; ++c) {
+#pragma unroll
+                                for (int e = 0; e < 32; ++e)
+                                    raw[c][e] = __float_as_uint(__uint_as_float(raw[c][e]) * alpha);
+                                tc::tmem_st32(tmem + lane_off + 2 * kTileN + (c0 + c) * 32, raw[c]);
+                            }
                         }
                         tc::tmem_wait_st();
                         if (need) {
@@ -516,29 +557,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-                // probabilities, packed to bf16 pairs
-                uint32_t pk[kTileN / 2];
-                float lsum = 0.f;
+                // probabilities, packed to bf16 pairs and written to P one 64-key
+                // block at a time: chunk c of a 128-byte row lands at chunk c ^ (row % 8)
+                float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int c = 0; c < kTileN; c += 2) {
-                    const float p0v = fast_exp2(fmaf(sv[c], p.scale_log2, -m));
-                    const float p1v = fast_exp2(fmaf(sv[c + 1], p.scale_log2, -m));
-                    lsum += p0v + p1v;
-                    pk[c / 2] = pack_bf16x2(p0v, p1v);
-                }
-                l += lsum;
-                if (T > 0) NPV_WAIT(p_empty, (T - 1) & 1);  // P buffer free again
-                // row `row` of P, K-major with the 128-byte swizzle: 16-byte chunk c of
-                // a 128-byte row lands at chunk c ^ (row % 8)
-                {
-                    uint8_t *prow = sP + row * 128;
+                for (int kb = 0; kb < kTileN / 64; ++kb) {
+                    uint32_t pk[32];
 #pragma unroll
-                    for (int c = 0; c < kTileN / 8; ++c) {
-                        const int kb = c >> 3, ch = c & 7;
-                        uint4 v4 = make_uint4(pk[c * 4 + 0], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
-                        *reinterpret_cast<uint4 *>(prow + kb * (kTileM * 128) + ((ch ^ (row & 7)) * 16)) = v4;
+                    for (int c = 0; c < 64; c += 2) {
+                        const float p0v = fast_exp2(fmaf(sv[kb * 64 + c], p.scale_log2, -m));
+                        const float p1v = fast_exp2(fmaf(sv[kb * 64 + c + 1], p.scale_log2, -m));
+                        ls8[(c / 2) & 7] += p0v + p1v;
+                        pk[c / 2] = pack_bf16x2(p0v, p1v);
+                    }
+                    if (kb == 0 && T > 0) NPV_WAIT(p_empty, (T - 1) & 1);  // P buffer free again
+                    uint8_t *prow = sP + kb * (kTileM * 128) + row * 128;
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        uint4 v4 = make_uint4(pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
+                        *reinterpret_cast<uint4 *>(prow + ((ch ^ (row & 7)) * 16)) = v4;
                     }
                 }
+                l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
                 tc::fence_proxy_async_smem();
                 tc::fence_before_sync();
                 __syncwarp();
@@ -551,18 +591,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float inv = 1.0f / l;
                 uint16_t *orow = p.out + ((int64_t)(it.row0 + it.p0 + pos) * p.num_q_heads + it.h * G + jh) * D;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t raw[32];
-                    tc::tmem_ld32(tmem + lane_off + 2 * kTileN + c * 32, raw);
+                for (int c0 = 0; c0 < D / 32; c0 += 2) {
+                    uint32_t raw[2][32];
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) tc::tmem_ld32(tmem + lane_off + 2 * kTileN + (c0 + c) * 32, raw[c]);
                     tc::tmem_wait_ld();
                     if (valid_row) {
 #pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            float f[8];
+                        for (int c = 0; c < 2; ++c)
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(raw[v * 8 + e]) * inv;
-                            st_global_v4(orow + c * 32 + v * 8, pack8(f));
-                        }
+                            for (int v = 0; v < 4; ++v) {
+                                float f[8];
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(raw[c][v * 8 + e]) * inv;
+                                st_global_v4(orow + (c0 + c) * 32 + v * 8, pack8(f));
+                            }
                     }
                 }
             }

@@ -64,6 +64,9 @@ def lib() -> C.CDLL:
     l.npv_paged_decode_attention.argtypes = [p, p, i64, p, p, p, i32, p, i32, i32, i32, i32, i32, i32, C.c_float,
                                              p, sz, p]
     l.npv_paged_decode_attention.restype = C.c_int
+    l.npv_store_kvcache_and_decode_attention.argtypes = [p, p, i64, p, p, i64, i64, p, p, p, p, i32, p, i32, i32,
+                                                         i32, i32, i32, i32, C.c_float, p, sz, p]
+    l.npv_store_kvcache_and_decode_attention.restype = C.c_int
     l.npv_paged_prefill_workspace_size.argtypes = [i32, i32, i32, i32, i32]
     l.npv_paged_prefill_workspace_size.restype = sz
     l.npv_paged_prefill_attention.argtypes = [p, p, p, i32, i32, p, p, p, i32, p, i32, i32, i32, i32, i32, i32,
@@ -138,6 +141,31 @@ def paged_decode_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
                                             _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), B, Hq,
                                             Hkv, D, NB, BS, float(scale or 0.0), _ptr(workspace),
                                             workspace.numel(), _stream(stream)), "npv_paged_decode_attention")
+    return out
+
+
+def store_kvcache_and_decode_attention(q: torch.Tensor, key: torch.Tensor, value: torch.Tensor,
+                                       k_cache: torch.Tensor, v_cache: torch.Tensor, slot_mapping: torch.Tensor,
+                                       block_tables: torch.Tensor, context_lens: torch.Tensor,
+                                       scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                                       workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One decode step in one launch set: store key/value [B, Hkv, D] at slot_mapping [B], then
+    decode attention for q [B, Hq, D] -> out [B, Hq, D]."""
+    NB, BS, Hkv, D = _cache_shape(k_cache)
+    B, Hq, Dq = q.shape
+    assert Dq == D and q.stride(2) == 1 and q.stride(1) == D
+    assert key.shape == (B, Hkv, D) and value.shape == (B, Hkv, D) and slot_mapping.shape == (B,)
+    assert key.stride(-1) == 1 and key.stride(-2) == D and value.stride(-1) == 1 and value.stride(-2) == D
+    assert slot_mapping.dtype == torch.int32 and block_tables.dtype == torch.int32 and block_tables.is_contiguous()
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=q.dtype, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(decode_workspace_size(B, Hq, Hkv, D), q.device)
+    _check(lib().npv_store_kvcache_and_decode_attention(
+        _ptr(out), _ptr(q), q.stride(0), _ptr(key), _ptr(value), key.stride(0), value.stride(0), _ptr(slot_mapping),
+        _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), B, Hq, Hkv, D,
+        NB, BS, float(scale or 0.0), _ptr(workspace), workspace.numel(), _stream(stream)),
+        "npv_store_kvcache_and_decode_attention")
     return out
 
 
