@@ -107,6 +107,52 @@ def profiled_traffic(workload: str):
 
 
 # ---------------------------------------------------------------------------
+# ranks: one process per GPU; timing is a max over ranks, work a sum
+# ---------------------------------------------------------------------------
+
+class Ranks:
+    """Barrier and reductions over the job's ranks (NCCL on GPUs, gloo on CPU).
+
+    The data path has no collective: each rank runs its own replica of the
+    workload; only timings and counts cross ranks."""
+
+    def __init__(self, world: int, device=None):
+        self.world = world
+        self.device = device
+
+    def _dist(self):
+        import torch.distributed as dist
+
+        return dist
+
+    def barrier(self):
+        if self.world > 1:
+            self._dist().barrier()
+
+    def _reduce(self, x: float, op) -> float:
+        if self.world == 1:
+            return float(x)
+        import torch
+
+        t = torch.tensor([float(x)], dtype=torch.float64, device=self.device)
+        self._dist().all_reduce(t, op=op)
+        return float(t.item())
+
+    def max(self, x: float) -> float:
+        return self._reduce(x, self._dist().ReduceOp.MAX) if self.world > 1 else float(x)
+
+    def sum(self, x: float) -> float:
+        return self._reduce(x, self._dist().ReduceOp.SUM) if self.world > 1 else float(x)
+
+
+def whole_job_rate(ranks: Ranks, local_units: float, local_ms: float) -> tuple:
+    """(units of all ranks per second, slowest rank's ms): the job is as fast as its slowest rank."""
+    ms = ranks.max(local_ms)
+    units = ranks.sum(local_units)
+    return units / (ms * 1e-3), ms
+
+
+# ---------------------------------------------------------------------------
 # workload bookkeeping (host side)
 # ---------------------------------------------------------------------------
 
@@ -349,16 +395,9 @@ def npv_arm(args, rank, world, local_rank):
 
     launches_per_step = (5 if mixed else (3 if args.separate_store else 2))
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks(world, dev)
+    barrier = ranks.barrier
+    max_over_ranks = ranks.max
 
     bytes_steps = [step_bytes(wl, i % nsteps) for i in range(args.steps)]
     store_bytes = sum(b[0] for b in bytes_steps)
@@ -424,8 +463,9 @@ def npv_arm(args, rank, world, local_rank):
         e2e = npv_e2e(args, wl, st, ws, dev, stream, ops, W, barrier, max_over_ranks, step_fn_kind(args, mixed))
 
     peak, peak_kind = measured_peaks()
-    total_bytes = (store_bytes + attn_bytes) * world
-    value = total_bytes / (ms * 1e-3) / 1e9
+    # value: bytes of all ranks over the slowest rank's time (ms is already the max)
+    rate, _ = whole_job_rate(ranks, store_bytes + attn_bytes, ms)
+    value = rate / 1e9
     call_bytes = attn_bytes / args.steps + (0 if (mixed or args.separate_store) else store_bytes / args.steps)
     achieved = call_bytes / (call_ms * 1e-3) / 1e9
     line = {
@@ -433,7 +473,7 @@ def npv_arm(args, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(wl),
-        "tokens_per_s": world * args.steps * wl.total_q / (ms * 1e-3),
+        "tokens_per_s": ranks.sum(args.steps * wl.total_q) / (ms * 1e-3),
         "pct_of_peak_hbm": 100.0 * value / world / peak,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
