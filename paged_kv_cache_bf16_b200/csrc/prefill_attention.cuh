@@ -18,18 +18,24 @@
 //     contiguous (so the items that read the same K/V run at the same time and
 //     share it through L2).  The persistent main kernel (one CTA per SM) takes
 //     items (pair, KV head) from that list in snake order.
-//   * Warp roles: warp 4 issues the TMA loads of Q (once per item) and of the
-//     K tiles (128 keys) through a 3-stage ring, warp 6 those of the V tiles
-//     through a 2-stage ring; block ids come from the block table a 32-entry
-//     window at a time, one TMA box per block piece.  A K stage is released as
-//     soon as its S = Q K^T product completes, so K loads run ahead of the P.V
-//     products.  Warp 5 owns tensor memory and issues tcgen05.mma from one
-//     thread; warps 0-3 run the softmax, one TMEM lane (= one query row) per
-//     thread.
-//   * Tensor memory holds S twice (so S for tile j+1 is computed while the
-//     softmax reads tile j) and the O accumulator.  S = Q K^T reads Q and K as
-//     K-major 128-byte-swizzled operands; O += P V reads P (bf16, written by the
-//     softmax threads in the same swizzle) as K-major and V as MN-major.
+//   * Operands: an M128 x N128 x K16 tcgen05.mma with both operands in shared
+//     memory reads 8 KB per 64 cycles, the whole shared-memory bandwidth of the
+//     tensor path, so anything else in shared memory slows the MMAs.  Q and P
+//     therefore live in tensor memory (the A operand of both products): Q is
+//     written there once per item by the softmax threads straight from global
+//     memory, P by the softmax threads after the exponentials.  Shared memory
+//     carries only K and V: TMA writes them, the MMAs read them.
+//   * Warp roles: warp 8 issues the TMA loads of the K tiles (128 keys) through
+//     a 3-stage ring, warp 10 those of the V tiles through a 3-stage ring; block
+//     ids come from the block table a 32-entry window at a time, one TMA box per
+//     block piece.  A K stage is released as soon as S = Q K^T completes.  Warp 9
+//     owns tensor memory and issues tcgen05.mma from one thread.  Two softmax
+//     warpgroups (warps 0-3 and 4-7) each take 64 of the 128 key columns of every
+//     S tile, one TMEM lane (= one query row) per thread, and exchange per-row
+//     partial maxima and sums through shared memory guarded by mbarriers.
+//   * Tensor memory (512 columns): S double-buffered (2 x 128 fp32), O (D fp32),
+//     Q (D/2 columns of bf16 pairs), P (64 columns of bf16 pairs).  K is read as
+//     a K-major 128-byte-swizzled operand, V as MN-major.
 //   * The softmax keeps a per-row running max in the log2 domain and rescales
 //     the O accumulator only when the max grows by more than 2^8 (otherwise the
 //     stale max is kept; the final division by the row sum corrects it exactly
@@ -46,12 +52,17 @@ namespace prefill {
 constexpr int kTileM = 128;   // query rows per item (MMA M)
 constexpr int kTileN = 128;   // keys per KV tile (MMA N of S, K of P.V)
 constexpr int kKStages = 3;   // K ring depth (a K stage is free once S = Q K^T is done)
-constexpr int kVStages = 2;   // V ring depth (a V stage is free once O += P V is done)
-constexpr int kThreads = 224; // 4 softmax warps, K producer, MMA, V producer
-constexpr int kKProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kVProducerWarp = 6;
+constexpr int kVStages = 3;   // V ring depth (a V stage is free once O += P V is done)
+constexpr int kThreads = 352; // 8 softmax warps, K producer, MMA, V producer
+constexpr int kSoftmaxWarps = 8;
+constexpr int kKProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kVProducerWarp = 10;
+constexpr int kHalf = kTileN / 2;  // key columns of an S tile per softmax warpgroup
 constexpr int kTmemCols = 512;
+constexpr int kTmemO = 2 * kTileN;  // O: [256, 256 + D)
+constexpr int kTmemQ = 384;         // Q: [384, 384 + D/2), bf16 pairs
+constexpr int kTmemP = 448;         // P: [448, 512), bf16 pairs
 constexpr int kBuckets = 4096;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -68,24 +79,24 @@ struct Params {
     int32_t block_size;
     int32_t max_blocks_per_seq;
     int32_t box_tokens;  // tokens per K/V TMA box: 128 when block_size % 128 == 0, else 16
+    const uint16_t *q;   // [total_q, Hq, D]
     float scale_log2;
     int32_t *plan_count;  // [1]: number of (sequence, row-tile) pairs
     int2 *plan_pairs;     // [max_pairs]: (sequence, row tile), longest first
     int32_t max_pairs;
 };
 
-// Shared-memory layout (bytes from a 1024-aligned base).
+// Shared-memory layout (bytes from a 1024-aligned base): barriers and the
+// softmax warpgroups' exchange slots, then the K and V rings.
 template <int D>
 struct Smem {
-    static constexpr int kHeader = 1024;
-    static constexpr int kQ = kTileM * D * 2;
+    static constexpr int kHeader = 4096;
+    static constexpr int kXmax = 512;    // float [2 parity][2 warpgroups][128 rows]
+    static constexpr int kXsum = 2560;   // float [2 warpgroups][128 rows]
     static constexpr int kKV = kTileN * D * 2;
-    static constexpr int kP = kTileM * kTileN * 2;
-    static constexpr int q = kHeader;
-    static constexpr int k = q + kQ;
+    static constexpr int k = kHeader;
     static constexpr int v = k + kKStages * kKV;
-    static constexpr int p = v + kVStages * kKV;
-    static constexpr int total = p + kP;
+    static constexpr int total = v + kVStages * kKV;
 };
 
 // Per-item quantities every warp role derives the same way.
@@ -272,38 +283,40 @@ __device__ __forceinline__ int tile_boxes(const Params &p, const Item &it, const
 
 template <int D, int G>
 __global__ void __launch_bounds__(kThreads, 1)
-    prefill_attention_kernel(const Params p, const __grid_constant__ CUtensorMap qmap,
-                             const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap) {
+    prefill_attention_kernel(const Params p, const __grid_constant__ CUtensorMap kmap,
+                             const __grid_constant__ CUtensorMap vmap) {
     using L = Smem<D>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 128-byte-swizzled tiles need 1024-byte-aligned shared addresses
     uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
-    uint64_t *q_full = bars + 0;
-    uint64_t *q_empty = bars + 1;
-    uint64_t *k_full = bars + 2;     // [kKStages]
-    uint64_t *k_empty = bars + 5;    // [kKStages]
-    uint64_t *v_full = bars + 8;     // [kVStages]
-    uint64_t *v_empty = bars + 10;   // [kVStages]
-    uint64_t *s_full = bars + 12;    // [2]
-    uint64_t *s_free = bars + 14;    // [2]
-    uint64_t *p_full = bars + 16;
-    uint64_t *p_empty = bars + 17;
-    uint64_t *o_full = bars + 18;
-    uint64_t *o_free = bars + 19;
-    uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(bars + 20);
-    int *abort_flag = reinterpret_cast<int *>(bars + 21);
-    uint8_t *sQ = smem + L::q;
+    uint64_t *q_full = bars + 0;   // Q of the item is in tensor memory (8 softmax warps)
+    uint64_t *q_empty = bars + 1;  // the item's last S product is done
+    uint64_t *k_full = bars + 2;   // [kKStages]
+    uint64_t *k_empty = bars + 5;  // [kKStages]
+    uint64_t *v_full = bars + 8;   // [kVStages]
+    uint64_t *v_empty = bars + 11; // [kVStages]
+    uint64_t *s_full = bars + 14;  // [2]
+    uint64_t *s_free = bars + 16;  // [2]
+    uint64_t *p_full = bars + 18;
+    uint64_t *p_empty = bars + 19;
+    uint64_t *o_full = bars + 20;
+    uint64_t *o_free = bars + 21;
+    uint64_t *x_full = bars + 22;  // [2]: partial row maxima exchanged, by tile parity
+    uint64_t *l_full = bars + 24;  // partial row sums exchanged (once per item)
+    uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(bars + 25);
+    int *abort_flag = reinterpret_cast<int *>(bars + 26);
+    float *xmax = reinterpret_cast<float *>(smem + L::kXmax);
+    float *xsum = reinterpret_cast<float *>(smem + L::kXsum);
     uint8_t *sK = smem + L::k;
     uint8_t *sV = smem + L::v;
-    uint8_t *sP = smem + L::p;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int kDBlocks = D / 64;        // 64-element (128-byte) column blocks
-    constexpr int kBlockBytes = kTileN * 128;  // one column block of a 128-row tile
+    constexpr int kDBlocks = D / 64;            // 64-element (128-byte) column blocks
+    constexpr int kBlockBytes = kTileN * 128;   // one column block of a 128-row K or V tile
 
     if (threadIdx.x == 0) {
-        mbar_init(q_full, 1);
+        mbar_init(q_full, kSoftmaxWarps);
         mbar_init(q_empty, 1);
         for (int s = 0; s < kKStages; ++s) {
             mbar_init(&k_full[s], 1);
@@ -315,17 +328,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&s_full[s], 1);
-            mbar_init(&s_free[s], 4);
+            mbar_init(&s_free[s], kSoftmaxWarps);
+            mbar_init(&x_full[s], kSoftmaxWarps);
         }
-        mbar_init(p_full, 4);
+        mbar_init(p_full, kSoftmaxWarps);
         mbar_init(p_empty, 1);
         mbar_init(o_full, 1);
-        mbar_init(o_free, 4);
+        mbar_init(o_free, kSoftmaxWarps);
+        mbar_init(l_full, kSoftmaxWarps);
         *abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == kKProducerWarp && lane == 0) {
-        tc::prefetch_tensormap(&qmap);
         tc::prefetch_tensormap(&kmap);
         tc::prefetch_tensormap(&vmap);
     }
@@ -350,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint64_t *empty = is_k ? k_empty : v_empty;
         uint8_t *ring = is_k ? sK : sV;
         const CUtensorMap *map = is_k ? &kmap : &vmap;
-        uint32_t q_iter = 0, kv_iter = 0;
+        uint32_t kv_iter = 0;
         const int BS = p.block_size;
         for (long long r = 0; r < rounds; ++r) {
             const long long idx = item_index(r);
@@ -358,16 +372,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Item it = load_item<G>(p, idx);
             const int32_t *bt_row = p.block_tables + (size_t)it.b * p.max_blocks_per_seq;
             int win = -1, win_val = -1;
-            if (is_k) {
-                NPV_WAIT(q_empty, (q_iter & 1) ^ 1);
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(q_full, (uint32_t)L::kQ);
-                    for (int db = 0; db < kDBlocks; ++db)
-                        tc::tma_load_3d(sQ + db * (kTileM * 128), &qmap, db * 64, it.h * G, it.row0 + it.p0,
-                                        q_full);
-                }
-                ++q_iter;
-            }
             for (int t = 0; t < it.ntiles; ++t, ++kv_iter) {
                 const int s = (int)(kv_iter % nstages);
                 NPV_WAIT(&empty[s], ((kv_iter / nstages) & 1) ^ 1);
@@ -397,21 +401,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ============================ MMA issuer ============================
         constexpr uint32_t idesc_s = tc::idesc_bf16_f32(kTileM, kTileN, 0, 0);
         constexpr uint32_t idesc_o = tc::idesc_bf16_f32(kTileM, D, 0, 1);
-        const uint32_t q_addr = smem_addr(sQ), k_addr = smem_addr(sK), v_addr = smem_addr(sV),
-                       p_addr = smem_addr(sP);
-        uint32_t q_iter = 0, kv_iter = 0, item_iter = 0;
+        const uint32_t k_addr = smem_addr(sK), v_addr = smem_addr(sV);
+        uint32_t kv_iter = 0, item_iter = 0;
         for (long long r = 0; r < rounds; ++r) {
             const long long idx = item_index(r);
             if (idx >= n_items) continue;
             const Item it = load_item<G>(p, idx);
-            NPV_WAIT(q_full, q_iter & 1);
-            ++q_iter;
+            NPV_WAIT(q_full, item_iter & 1);
             tc::fence_after_sync();
             for (int t = 0; t <= it.ntiles; ++t) {
                 if (t < it.ntiles) {
-                    // ---- S[t % 2] = Q K_t^T
+                    // ---- S[t % 2] = Q K_t^T  (Q from tensor memory)
                     const uint32_t T = kv_iter + t;
-                    const int s = T & 1;              // S buffer
+                    const int s = T & 1;                 // S buffer
                     const int ks = (int)(T % kKStages);  // K stage
                     NPV_WAIT(&k_full[ks], (T / kKStages) & 1);
                     NPV_WAIT(&s_free[s], ((T >> 1) & 1) ^ 1);
@@ -420,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int k = 0; k < D / 16; ++k) {
                             const uint32_t off = (k >> 2) * kBlockBytes + (k & 3) * 32;
-                            tc::mma_bf16_ss(tmem + s * kTileN, tc::smem_desc_sw128(q_addr + off, 16, 1024),
+                            tc::mma_bf16_ts(tmem + s * kTileN, tmem + kTmemQ + k * 8,
                                             tc::smem_desc_sw128(k_addr + ks * L::kKV + off, 16, 1024), idesc_s,
                                             k > 0);
                         }
@@ -431,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     __syncwarp();
                 }
                 if (t > 0) {
-                    // ---- O (+)= P_{t-1} V_{t-1}
+                    // ---- O (+)= P_{t-1} V_{t-1}  (P from tensor memory)
                     const int tp = t - 1;
                     const uint32_t T = kv_iter + tp;
                     const int s = (int)(T % kVStages);  // V stage
@@ -457,9 +459,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::fence_after_sync();
                     if (lane == 0) {
                         for (int k = 0; k < ksteps; ++k) {
-                            const uint32_t poff = (k >> 2) * (kTileM * 128) + (k & 3) * 32;
                             const uint32_t voff = k * 16 * 128;
-                            tc::mma_bf16_ss(tmem + 2 * kTileN, tc::smem_desc_sw128(p_addr + poff, 16, 1024),
+                            tc::mma_bf16_ts(tmem + kTmemO, tmem + kTmemP + k * 8,
                                             tc::smem_desc_sw128(v_addr + s * L::kKV + voff, kBlockBytes, 1024),
                                             idesc_o, tp > 0 || k > 0);
                         }
@@ -474,9 +475,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++item_iter;
         }
     } else {
-        // ============================ softmax (warps 0-3) ============================
-        const int row = warp * 32 + lane;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        // ======== softmax: warpgroup wg (warps 4 wg .. 4 wg + 3) owns key columns [64 wg, 64 wg + 64) ========
+        const int wg = warp >> 2;
+        const int row = (warp & 3) * 32 + lane;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const int kc0 = wg * kHalf;    // first key column of this warpgroup
+        const int oc0 = wg * (D / 2);  // first O column (and first Q element) of this warpgroup
         uint32_t kv_iter = 0, item_iter = 0;
         for (long long r = 0; r < rounds; ++r) {
             const long long idx = item_index(r);
@@ -486,69 +490,99 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool valid_row = pos < it.npos;
             const int lim = valid_row ? (it.L - it.n + it.p0 + pos) : (it.L - 1);
             const int lim_min = it.L - it.n + it.p0;  // smallest limit among the tile's rows
+            {
+                // ---- Q row -> tensor memory: this warpgroup's half of the row's D elements
+                uint32_t qw[D / 4];
+                if (valid_row) {
+                    const uint16_t *qrow =
+                        p.q + ((int64_t)(it.row0 + it.p0 + pos) * p.num_q_heads + it.h * G + jh) * D + oc0;
+#pragma unroll
+                    for (int v = 0; v < D / 16; ++v) {
+                        const uint4 x = ld_nc_v4(qrow + v * 8);
+                        qw[v * 4 + 0] = x.x;
+                        qw[v * 4 + 1] = x.y;
+                        qw[v * 4 + 2] = x.z;
+                        qw[v * 4 + 3] = x.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int v = 0; v < D / 4; ++v) qw[v] = 0u;
+                }
+                NPV_WAIT(q_empty, (item_iter & 1) ^ 1);  // the previous item's S products are done
+                tc::fence_after_sync();
+                if constexpr (D == 128) {
+                    tc::tmem_st32(tmem + lane_off + kTmemQ + wg * 32, qw);
+                } else {
+                    tc::tmem_st16(tmem + lane_off + kTmemQ + wg * 16, qw);
+                }
+                tc::tmem_wait_st();
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(q_full);
+            }
             float m = -INFINITY, l = 0.f;
             for (int t = 0; t < it.ntiles; ++t) {
                 const uint32_t T = kv_iter + t;
                 const int sb = T & 1;
                 NPV_WAIT(&s_full[sb], (T >> 1) & 1);
                 tc::fence_after_sync();
-                float sv[kTileN];
+                float sv[kHalf];
                 {
-                    // all four TMEM loads in flight before a single wait
-                    uint32_t raw[kTileN / 32][32];
+                    uint32_t raw[kHalf / 32][32];
 #pragma unroll
-                    for (int c = 0; c < kTileN / 32; ++c) tc::tmem_ld32(tmem + lane_off + sb * kTileN + c * 32, raw[c]);
+                    for (int c = 0; c < kHalf / 32; ++c)
+                        tc::tmem_ld32(tmem + lane_off + sb * kTileN + kc0 + c * 32, raw[c]);
                     tc::tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < kTileN / 32; ++c)
+                    for (int c = 0; c < kHalf / 32; ++c)
 #pragma unroll
                         for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(raw[c][e]);
                 }
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s_free[sb]);
-                const int kv0 = t * kTileN;
-                if (kv0 + kTileN - 1 > lim_min) {
+                const int kv0 = t * kTileN + kc0;
+                if (kv0 + kHalf - 1 > lim_min) {
 #pragma unroll
-                    for (int c = 0; c < kTileN; ++c)
+                    for (int c = 0; c < kHalf; ++c)
                         if (kv0 + c > lim) sv[c] = -INFINITY;
                 }
-                // row max with 8 independent chains
                 float mx8[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) mx8[e] = sv[e];
 #pragma unroll
-                for (int c = 8; c < kTileN; c += 8)
+                for (int c = 8; c < kHalf; c += 8)
 #pragma unroll
                     for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], sv[c + e]);
-                const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-                const float m_tile = mx * p.scale_log2;
+                const float pmax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+                // full-row max: swap partial maxima with the other warpgroup
+                xmax[(sb * 2 + wg) * kTileM + row] = pmax;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&x_full[sb]);
+                NPV_WAIT(&x_full[sb], (T >> 1) & 1);
+                const float omax = xmax[(sb * 2 + (1 - wg)) * kTileM + row];
+                const float m_tile = fmaxf(pmax, omax) * p.scale_log2;
                 if (t == 0) {
                     m = m_tile;
                 } else {
                     const float m_new = fmaxf(m, m_tile);
-                    const bool need = m_new > m + kRescaleThreshold;
+                    const bool need = m_new > m + kRescaleThreshold;  // the same in both warpgroups
                     if (__any_sync(0xffffffffu, need)) {
                         // the previous P.V must have landed before O is rescaled
                         NPV_WAIT(p_empty, (T - 1) & 1);
                         tc::fence_after_sync();
                         const float alpha = need ? fast_exp2(m - m_new) : 1.0f;
-                        // 32 columns at a time: the scores are still live in registers
+                        // this warpgroup's half of O, 32 columns at a time
 #pragma unroll
-                        for (int c0 = 0; c0 < D / 32; c0 += 1) {
-                            uint32_t raw[1][32];
-#pragma unroll
-                            for (int c = 0; c < 1; ++c)
-                                tc::tmem_ld32(tmem + lane_off + 2 * kTileN + (c0 + c) * 32, raw[c]);
+                        for (int c = 0; c < D / 64; ++c) {
+                            uint32_t raw[32];
+                            const uint32_t ta = tmem + lane_off + kTmemO + oc0 + c * 32;
+                            tc::tmem_ld32(ta, raw);
                             tc::tmem_wait_ld();
 #pragma unroll
-                            for (int c = 0; c < 1; ++c) {
-#pragma unroll
-                                for (int e = 0; e < 32; ++e)
-                                    raw[c][e] = __float_as_uint(__uint_as_float(raw[c][e]) * alpha);
-                                tc::tmem_st32(tmem + lane_off + 2 * kTileN + (c0 + c) * 32, raw[c]);
-                            }
+                            for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
+                            tc::tmem_st32(ta, raw);
                         }
                         tc::tmem_wait_st();
                         if (need) {
@@ -557,56 +591,52 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-                // probabilities, packed to bf16 pairs and written to P one 64-key
-                // block at a time: chunk c of a 128-byte row lands at chunk c ^ (row % 8)
+                // probabilities of this warpgroup's 64 keys, packed to bf16 pairs, into P's
+                // columns [32 wg, 32 wg + 32) of tensor memory
                 float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                uint32_t pk[kHalf / 2];
 #pragma unroll
-                for (int kb = 0; kb < kTileN / 64; ++kb) {
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int c = 0; c < 64; c += 2) {
-                        const float p0v = fast_exp2(fmaf(sv[kb * 64 + c], p.scale_log2, -m));
-                        const float p1v = fast_exp2(fmaf(sv[kb * 64 + c + 1], p.scale_log2, -m));
-                        ls8[(c / 2) & 7] += p0v + p1v;
-                        pk[c / 2] = pack_bf16x2(p0v, p1v);
-                    }
-                    if (kb == 0 && T > 0) NPV_WAIT(p_empty, (T - 1) & 1);  // P buffer free again
-                    uint8_t *prow = sP + kb * (kTileM * 128) + row * 128;
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        uint4 v4 = make_uint4(pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
-                        *reinterpret_cast<uint4 *>(prow + ((ch ^ (row & 7)) * 16)) = v4;
-                    }
+                for (int c = 0; c < kHalf; c += 2) {
+                    const float p0v = fast_exp2(fmaf(sv[c], p.scale_log2, -m));
+                    const float p1v = fast_exp2(fmaf(sv[c + 1], p.scale_log2, -m));
+                    ls8[(c / 2) & 7] += p0v + p1v;
+                    pk[c / 2] = pack_bf16x2(p0v, p1v);
                 }
                 l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
-                tc::fence_proxy_async_smem();
+                if (T > 0) NPV_WAIT(p_empty, (T - 1) & 1);  // the previous P.V has read P
+                tc::fence_after_sync();
+                tc::tmem_st32(tmem + lane_off + kTmemP + wg * (kHalf / 2), pk);
+                tc::tmem_wait_st();
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(p_full);
             }
-            // ---- epilogue: O / l -> bf16
+            // ---- epilogue: full row sum from the two partial sums, then O / l -> bf16
+            xsum[wg * kTileM + row] = l;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(l_full);
+            NPV_WAIT(l_full, item_iter & 1);
             NPV_WAIT(o_full, item_iter & 1);
             tc::fence_after_sync();
             {
-                const float inv = 1.0f / l;
-                uint16_t *orow = p.out + ((int64_t)(it.row0 + it.p0 + pos) * p.num_q_heads + it.h * G + jh) * D;
+                const float lo = xsum[(1 - wg) * kTileM + row];
+                uint32_t raw[D / 64][32];
 #pragma unroll
-                for (int c0 = 0; c0 < D / 32; c0 += 2) {
-                    uint32_t raw[2][32];
+                for (int c = 0; c < D / 64; ++c) tc::tmem_ld32(tmem + lane_off + kTmemO + oc0 + c * 32, raw[c]);
+                tc::tmem_wait_ld();
+                const float inv = 1.0f / (l + lo);
+                uint16_t *orow =
+                    p.out + ((int64_t)(it.row0 + it.p0 + pos) * p.num_q_heads + it.h * G + jh) * D + oc0;
+                if (valid_row) {
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) tc::tmem_ld32(tmem + lane_off + 2 * kTileN + (c0 + c) * 32, raw[c]);
-                    tc::tmem_wait_ld();
-                    if (valid_row) {
+                    for (int c = 0; c < D / 64; ++c)
 #pragma unroll
-                        for (int c = 0; c < 2; ++c)
+                        for (int v = 0; v < 4; ++v) {
+                            float f[8];
 #pragma unroll
-                            for (int v = 0; v < 4; ++v) {
-                                float f[8];
-#pragma unroll
-                                for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(raw[c][v * 8 + e]) * inv;
-                                st_global_v4(orow + (c0 + c) * 32 + v * 8, pack8(f));
-                            }
-                    }
+                            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(raw[c][v * 8 + e]) * inv;
+                            st_global_v4(orow + c * 32 + v * 8, pack8(f));
+                        }
                 }
             }
             tc::fence_before_sync();
