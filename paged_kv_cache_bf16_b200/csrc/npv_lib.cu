@@ -262,8 +262,8 @@ npv_status prefill_config(int32_t num_seqs, int32_t total_q, int num_q_heads, in
 }
 
 template <int D, int G>
-cudaError_t launch_prefill(const npv::prefill::Params &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
-                           const PrefillConfig &cfg, cudaStream_t stream) {
+cudaError_t launch_prefill(const npv::prefill::Params &p, const CUtensorMap &qmap, const CUtensorMap &kmap,
+                           const CUtensorMap &vmap, const PrefillConfig &cfg, cudaStream_t stream) {
     cudaError_t e = launch_pdl(npv::prefill::prefill_plan_kernel<G>, dim3(1), dim3(1024), 0, stream, p, D);
     if (e != cudaSuccess) return e;
     auto kernel = npv::prefill::prefill_attention_kernel<D, G>;
@@ -275,13 +275,14 @@ cudaError_t launch_prefill(const npv::prefill::Params &p, const CUtensorMap &kma
         if (e != cudaSuccess) return e;
         configured_smem[dev] = (int)cfg.smem;
     }
-    return launch_pdl(kernel, dim3(cfg.grid), dim3(npv::prefill::kThreads), cfg.smem, stream, p, kmap, vmap);
+    return launch_pdl(kernel, dim3(cfg.grid), dim3(npv::prefill::kThreads), cfg.smem, stream, p, qmap, kmap, vmap);
 }
 
-cudaError_t dispatch_prefill(int D, int G, const npv::prefill::Params &p, const CUtensorMap &kmap,
-                             const CUtensorMap &vmap, const PrefillConfig &cfg, cudaStream_t stream) {
+cudaError_t dispatch_prefill(int D, int G, const npv::prefill::Params &p, const CUtensorMap &qmap,
+                             const CUtensorMap &kmap, const CUtensorMap &vmap, const PrefillConfig &cfg,
+                             cudaStream_t stream) {
 #define NPV_PREFILL_CASE(DD, GG) \
-    if (D == DD && G == GG) return launch_prefill<DD, GG>(p, kmap, vmap, cfg, stream);
+    if (D == DD && G == GG) return launch_prefill<DD, GG>(p, qmap, kmap, vmap, cfg, stream);
     NPV_PREFILL_CASE(128, 1)
     NPV_PREFILL_CASE(128, 2)
     NPV_PREFILL_CASE(128, 4)
@@ -460,10 +461,13 @@ npv_status npv_paged_prefill_attention(void *out, const void *q, const int32_t *
     cudaStream_t s = (cudaStream_t)stream;
     const int D = head_dim, G = cfg.decode.group;
 
-    // tensor maps of the caches [NB * BS, Hkv, D], 128-byte swizzle (q is read directly)
-    CUtensorMap kmap, vmap;
+    // tensor maps, 128-byte swizzle: the caches [NB * BS, Hkv, D] in boxes of
+    // {64 elements, 1 head, box_tokens slots}; q [total_q, Hq, D] in boxes of
+    // {64 elements, G heads, 128 / G positions} (one 128-row tile of a KV head)
+    CUtensorMap qmap, kmap, vmap;
     const int box_tokens = (block_size % 128 == 0) ? 128 : 16;
-    if (!encode_map_3d(&kmap, k_cache, D, num_kv_heads, (uint64_t)num_blocks * block_size, 64, 1, box_tokens) ||
+    if (!encode_map_3d(&qmap, q, D, num_q_heads, (uint64_t)total_q, 64, G, npv::prefill::kTileM / G) ||
+        !encode_map_3d(&kmap, k_cache, D, num_kv_heads, (uint64_t)num_blocks * block_size, 64, 1, box_tokens) ||
         !encode_map_3d(&vmap, v_cache, D, num_kv_heads, (uint64_t)num_blocks * block_size, 64, 1, box_tokens))
         return NPV_ERR_CUDA;
 
@@ -488,7 +492,7 @@ npv_status npv_paged_prefill_attention(void *out, const void *q, const int32_t *
     p.plan_pairs = reinterpret_cast<int2 *>(ws + cfg.decode.ws_total + 256);
     p.max_pairs = cfg.max_pairs;
 
-    cudaError_t e = dispatch_prefill(D, G, p, kmap, vmap, cfg, s);
+    cudaError_t e = dispatch_prefill(D, G, p, qmap, kmap, vmap, cfg, s);
     if (e != cudaSuccess) return NPV_ERR_CUDA;
     // rows of sequences with exactly one query row: split-KV decode
     return run_decode(out, q, (int64_t)num_q_heads * head_dim, cu_seqlens_q, total_q, k_cache, v_cache,

@@ -18,29 +18,36 @@
 //     contiguous (so the items that read the same K/V run at the same time and
 //     share it through L2).  The persistent main kernel (one CTA per SM) takes
 //     items (pair, KV head) from that list in snake order.
-//   * Operands: an M128 x N128 x K16 tcgen05.mma with both operands in shared
-//     memory reads 8 KB per 64 cycles, the whole shared-memory bandwidth of the
-//     tensor path, so anything else in shared memory slows the MMAs.  Q and P
-//     therefore live in tensor memory (the A operand of both products): Q is
-//     written there once per item by the softmax threads straight from global
-//     memory, P by the softmax threads after the exponentials.  Shared memory
-//     carries only K and V: TMA writes them, the MMAs read them.
-//   * Warp roles: warp 8 issues the TMA loads of the K tiles (128 keys) through
-//     a 3-stage ring, warp 10 those of the V tiles through a 3-stage ring; block
-//     ids come from the block table a 32-entry window at a time, one TMA box per
-//     block piece.  A K stage is released as soon as S = Q K^T completes.  Warp 9
-//     owns tensor memory and issues tcgen05.mma from one thread.  Two softmax
-//     warpgroups (warps 0-3 and 4-7) each take 64 of the 128 key columns of every
-//     S tile, one TMEM lane (= one query row) per thread, and exchange per-row
-//     partial maxima and sums through shared memory guarded by mbarriers.
-//   * Tensor memory (512 columns): S double-buffered (2 x 128 fp32), O (D fp32),
-//     Q (D/2 columns of bf16 pairs), P (64 columns of bf16 pairs).  K is read as
-//     a K-major 128-byte-swizzled operand, V as MN-major.
+//   * Measured on B200: one tcgen05.mma M128 x N128 x K16 runs 64 cycles, but
+//     the issuing thread spends ~48 cycles per MMA instruction, ~50 per commit
+//     and ~58 per mbarrier wait.  One Q tile of 128 rows gives the issuer 16
+//     MMAs + 3 commits + 4 waits per 128-key tile, about the 1,024 cycles the
+//     tensor pipe needs for it, so the issuer's loop has no slack to spare: it
+//     issues S_{t+2} right after P_t V_t, and waits have a one-instruction fast
+//     path.
+//   * Split KV inside the CTA: softmax warpgroup j (warps 4-7, 8-11) takes the
+//     KV tiles T with T % 2 == j, with its own S buffer, running (max, sum) and
+//     O accumulator; the two partial results are merged in the epilogue.  The
+//     warpgroups never wait for each other inside the KV loop and their
+//     exponential phases interleave on the special-function units.
+//   * Warp roles: warp 0 owns tensor memory and issues tcgen05.mma from one
+//     thread; warp 1 issues the TMA loads of the K tiles (128 keys) through a
+//     3-stage ring, warp 2 those of the V tiles through a 2-stage ring (block ids
+//     from the block table a 32-entry window at a time, one TMA box per block
+//     piece); warp 3 loads each item's Q tile with one TMA box per 64 columns.
+//     The first warpgroup gives registers to the softmax warpgroups (setmaxnreg)
+//     so that a softmax thread holds a whole 128-key row of S.
+//   * Operands: S = Q K^T reads Q and K from shared memory (K-major, 128-byte
+//     swizzle); P V reads P from tensor memory, where the softmax writes it as
+//     bf16 pairs over the first 64 columns of its own S buffer, and V from
+//     shared memory (MN-major).  Tensor memory (512 columns): S_0, S_1 (128
+//     fp32 columns each), O_0, O_1 (D columns each).
 //   * The softmax keeps a per-row running max in the log2 domain and rescales
-//     the O accumulator only when the max grows by more than 2^8 (otherwise the
+//     its O accumulator only when the max grows by more than 2^8 (otherwise the
 //     stale max is kept; the final division by the row sum corrects it exactly
 //     in real arithmetic).  V rows past the context of the last tile are zeroed
-//     before the P.V product so unwritten cache slots never meet it.
+//     before the P.V product so unwritten cache slots never meet it; rows of the
+//     tile past its positions attend like its first row and are not stored.
 #pragma once
 
 #include "npv_device.cuh"
@@ -52,17 +59,16 @@ namespace prefill {
 constexpr int kTileM = 128;   // query rows per item (MMA M)
 constexpr int kTileN = 128;   // keys per KV tile (MMA N of S, K of P.V)
 constexpr int kKStages = 3;   // K ring depth (a K stage is free once S = Q K^T is done)
-constexpr int kVStages = 3;   // V ring depth (a V stage is free once O += P V is done)
-constexpr int kThreads = 352; // 8 softmax warps, K producer, MMA, V producer
+constexpr int kVStages = 2;   // V ring depth (a V stage is free once O += P V is done)
+constexpr int kThreads = 384;  // MMA, K producer, V producer, Q producer, 8 softmax warps
+constexpr int kMmaWarp = 0;
+constexpr int kKProducerWarp = 1;
+constexpr int kVProducerWarp = 2;
+constexpr int kQProducerWarp = 3;
+constexpr int kFirstSoftmaxWarp = 4;
 constexpr int kSoftmaxWarps = 8;
-constexpr int kKProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kVProducerWarp = 10;
-constexpr int kHalf = kTileN / 2;  // key columns of an S tile per softmax warpgroup
 constexpr int kTmemCols = 512;
-constexpr int kTmemO = 2 * kTileN;  // O: [256, 256 + D)
-constexpr int kTmemQ = 384;         // Q: [384, 384 + D/2), bf16 pairs
-constexpr int kTmemP = 448;         // P: [448, 512), bf16 pairs
+constexpr int kTmemO = 2 * kTileN;  // O_0 at [256, 256 + D), O_1 at [256 + D, 256 + 2 D)
 constexpr int kBuckets = 4096;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -87,14 +93,14 @@ struct Params {
 };
 
 // Shared-memory layout (bytes from a 1024-aligned base): barriers and the
-// softmax warpgroups' exchange slots, then the K and V rings.
+// warpgroups' (m, l) exchange, then the Q tile and the K and V rings.
 template <int D>
 struct Smem {
-    static constexpr int kHeader = 4096;
-    static constexpr int kXmax = 512;    // float [2 parity][2 warpgroups][128 rows]
-    static constexpr int kXsum = 2560;   // float [2 warpgroups][128 rows]
+    static constexpr int kHeader = 5120;
+    static constexpr int kXml = 1024;  // float2 [2 item parities][2 warpgroups][128 rows]
     static constexpr int kKV = kTileN * D * 2;
-    static constexpr int k = kHeader;
+    static constexpr int q = kHeader;
+    static constexpr int k = q + kTileM * D * 2;
     static constexpr int v = k + kKStages * kKV;
     static constexpr int total = v + kVStages * kKV;
 };
@@ -272,51 +278,72 @@ __device__ __forceinline__ int tile_boxes(const Params &p, const Item &it, const
     return nload;
 }
 
-#define NPV_WAIT(bar, parity)                     \
-    do {                                          \
-        if (!mbar_wait((bar), (parity))) {        \
-            *abort_flag = 1;                      \
-            goto finish;                          \
-        }                                         \
-        if (*(volatile int *)abort_flag) goto finish; \
+// Wait for the phase of `bar` with parity `parity`.  The fast path is a
+// single try_wait; the slow path also watches the CTA's abort flag (set by a
+// warp that gave up) and the time limit.  The outcome is made warp-uniform.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    bool ok = mbar_try_wait(bar, parity);
+    if (!ok) {
+        const uint64_t t0 = global_timer_ns();
+        for (uint32_t it = 1;; ++it) {
+            if (mbar_try_wait(bar, parity)) {
+                ok = true;
+                break;
+            }
+            if ((it & 15u) == 0) {
+                if (*abort_flag) break;
+                if (global_timer_ns() - t0 > kWaitLimitNs) {
+                    report_error(NPV_DEVERR_TIMEOUT);
+                    *abort_flag = 1;
+                    break;
+                }
+            }
+        }
+    }
+    return __all_sync(0xffffffffu, ok);
+}
+
+#define NPV_WAIT(bar, parity)                                   \
+    do {                                                        \
+        if (!wait_or_abort((bar), (parity), abort_flag)) goto finish; \
     } while (0)
+
+__device__ __forceinline__ void setmaxnreg_dec56() { asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory"); }
+__device__ __forceinline__ void setmaxnreg_inc224() { asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory"); }
 
 template <int D, int G>
 __global__ void __launch_bounds__(kThreads, 1)
-    prefill_attention_kernel(const Params p, const __grid_constant__ CUtensorMap kmap,
-                             const __grid_constant__ CUtensorMap vmap) {
+    prefill_attention_kernel(const Params p, const __grid_constant__ CUtensorMap qmap,
+                             const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap) {
     using L = Smem<D>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 128-byte-swizzled tiles need 1024-byte-aligned shared addresses
     uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
-    uint64_t *q_full = bars + 0;   // Q of the item is in tensor memory (8 softmax warps)
+    uint64_t *q_full = bars + 0;   // Q tile landed (TMA)
     uint64_t *q_empty = bars + 1;  // the item's last S product is done
     uint64_t *k_full = bars + 2;   // [kKStages]
-    uint64_t *k_empty = bars + 5;  // [kKStages]
-    uint64_t *v_full = bars + 8;   // [kVStages]
-    uint64_t *v_empty = bars + 11; // [kVStages]
-    uint64_t *s_full = bars + 14;  // [2]
-    uint64_t *s_free = bars + 16;  // [2]
-    uint64_t *p_full = bars + 18;
-    uint64_t *p_empty = bars + 19;
-    uint64_t *o_full = bars + 20;
-    uint64_t *o_free = bars + 21;
-    uint64_t *x_full = bars + 22;  // [2]: partial row maxima exchanged, by tile parity
-    uint64_t *l_full = bars + 24;  // partial row sums exchanged (once per item)
-    uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(bars + 25);
-    int *abort_flag = reinterpret_cast<int *>(bars + 26);
-    float *xmax = reinterpret_cast<float *>(smem + L::kXmax);
-    float *xsum = reinterpret_cast<float *>(smem + L::kXsum);
+    uint64_t *k_empty = bars + 2 + kKStages;
+    uint64_t *v_full = bars + 2 + 2 * kKStages;  // [kVStages]
+    uint64_t *v_empty = v_full + kVStages;
+    uint64_t *s_full = v_empty + kVStages;  // [2]: S tile in buffer j is ready
+    uint64_t *p_full = s_full + 2;          // [2]: P written over buffer j (4 warps of warpgroup j)
+    uint64_t *o_full = p_full + 2;          // the item's last P.V product is done
+    uint64_t *o_free = o_full + 1;          // both O accumulators read out (8 softmax warps)
+    uint64_t *ml_full = o_free + 1;         // per-row (m, l) of both warpgroups exchanged (8 softmax warps)
+    uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(ml_full + 1);
+    int *abort_flag = reinterpret_cast<int *>(ml_full + 2);
+    float2 *xml = reinterpret_cast<float2 *>(smem + L::kXml);  // [2 item parities][2 warpgroups][128 rows]
+    uint8_t *sQ = smem + L::q;
     uint8_t *sK = smem + L::k;
     uint8_t *sV = smem + L::v;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int kDBlocks = D / 64;            // 64-element (128-byte) column blocks
-    constexpr int kBlockBytes = kTileN * 128;   // one column block of a 128-row K or V tile
+    constexpr int kDBlocks = D / 64;           // 64-element (128-byte) column blocks
+    constexpr int kBlockBytes = kTileN * 128;  // one column block of a 128-row Q, K or V tile
 
     if (threadIdx.x == 0) {
-        mbar_init(q_full, kSoftmaxWarps);
+        mbar_init(q_full, 1);
         mbar_init(q_empty, 1);
         for (int s = 0; s < kKStages; ++s) {
             mbar_init(&k_full[s], 1);
@@ -326,20 +353,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&v_full[s], 1);
             mbar_init(&v_empty[s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&s_full[s], 1);
-            mbar_init(&s_free[s], kSoftmaxWarps);
-            mbar_init(&x_full[s], kSoftmaxWarps);
+        for (int j = 0; j < 2; ++j) {
+            mbar_init(&s_full[j], 1);
+            mbar_init(&p_full[j], kSoftmaxWarps / 2);
         }
-        mbar_init(p_full, kSoftmaxWarps);
-        mbar_init(p_empty, 1);
         mbar_init(o_full, 1);
         mbar_init(o_free, kSoftmaxWarps);
-        mbar_init(l_full, kSoftmaxWarps);
+        mbar_init(ml_full, kSoftmaxWarps);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == kKProducerWarp && lane == 0) {
+    if (warp == kQProducerWarp && lane == 0) {
+        tc::prefetch_tensormap(&qmap);
         tc::prefetch_tensormap(&kmap);
         tc::prefetch_tensormap(&vmap);
     }
@@ -356,8 +381,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     const long long n_items = (long long)p.plan_count[0] * p.num_kv_heads;
     const long long rounds = (n_items + gridDim.x - 1) / gridDim.x;
 
-    if (warp == kKProducerWarp || warp == kVProducerWarp) {
-        // ============================ TMA producers ============================
+    if (warp == kQProducerWarp) {
+        // ============================ Q tiles (TMA) ============================
+        setmaxnreg_dec56();
+        uint32_t item_iter = 0;
+        for (long long r = 0; r < rounds; ++r, ++item_iter) {
+            const long long idx = item_index(r);
+            if (idx >= n_items) break;
+            const Item it = load_item<G>(p, idx);
+            NPV_WAIT(q_empty, (item_iter & 1) ^ 1);  // the previous item's S products are done
+            if (lane == 0) {
+                mbar_arrive_expect_tx(q_full, (uint32_t)(kTileM * D * 2));
+                // rows (position, head) of the tile: box {64 elements, G heads, 128 / G positions}
+                for (int db = 0; db < kDBlocks; ++db)
+                    tc::tma_load_3d(sQ + db * kBlockBytes, &qmap, db * 64, it.h * G, it.row0 + it.p0, q_full);
+            }
+            __syncwarp();
+        }
+    } else if (warp == kKProducerWarp || warp == kVProducerWarp) {
+        // ============================ K / V tiles (TMA) ============================
+        setmaxnreg_dec56();
         const bool is_k = warp == kKProducerWarp;
         const int nstages = is_k ? kKStages : kVStages;
         uint64_t *full = is_k ? k_full : v_full;
@@ -368,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int BS = p.block_size;
         for (long long r = 0; r < rounds; ++r) {
             const long long idx = item_index(r);
-            if (idx >= n_items) continue;
+            if (idx >= n_items) break;
             const Item it = load_item<G>(p, idx);
             const int32_t *bt_row = p.block_tables + (size_t)it.b * p.max_blocks_per_seq;
             int win = -1, win_val = -1;
@@ -399,58 +442,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == kMmaWarp) {
         // ============================ MMA issuer ============================
+        setmaxnreg_dec56();
+        // Order within an item: S_0, S_1, then PV_t followed by S_{t+2}.  S_{t+2}
+        // overwrites the buffer that P_t occupies, which PV_t (issued before it
+        // by this thread) reads; tcgen05.mma ops of one thread run in order.
         constexpr uint32_t idesc_s = tc::idesc_bf16_f32(kTileM, kTileN, 0, 0);
         constexpr uint32_t idesc_o = tc::idesc_bf16_f32(kTileM, D, 0, 1);
-        const uint32_t k_addr = smem_addr(sK), v_addr = smem_addr(sV);
+        const uint64_t qdesc = tc::smem_desc_sw128(smem_addr(sQ), 16, 1024);
+        const uint64_t kdesc = tc::smem_desc_sw128(smem_addr(sK), 16, 1024);
+        const uint64_t vdesc = tc::smem_desc_sw128(smem_addr(sV), kBlockBytes, 1024);
         uint32_t kv_iter = 0, item_iter = 0;
         for (long long r = 0; r < rounds; ++r) {
             const long long idx = item_index(r);
-            if (idx >= n_items) continue;
+            if (idx >= n_items) break;
             const Item it = load_item<G>(p, idx);
             NPV_WAIT(q_full, item_iter & 1);
-            tc::fence_after_sync();
-            for (int t = 0; t <= it.ntiles; ++t) {
-                if (t < it.ntiles) {
-                    // ---- S[t % 2] = Q K_t^T  (Q from tensor memory)
+            for (int t = -2; t < it.ntiles; ++t) {
+                if (t >= 0) {
+                    // ---- O_j (+)= P_t V_t, j = T & 1 (P from tensor memory, over S_t)
                     const uint32_t T = kv_iter + t;
-                    const int s = T & 1;                 // S buffer
-                    const int ks = (int)(T % kKStages);  // K stage
-                    NPV_WAIT(&k_full[ks], (T / kKStages) & 1);
-                    NPV_WAIT(&s_free[s], ((T >> 1) & 1) ^ 1);
-                    tc::fence_after_sync();
-                    if (lane == 0) {
-#pragma unroll
-                        for (int k = 0; k < D / 16; ++k) {
-                            const uint32_t off = (k >> 2) * kBlockBytes + (k & 3) * 32;
-                            tc::mma_bf16_ts(tmem + s * kTileN, tmem + kTmemQ + k * 8,
-                                            tc::smem_desc_sw128(k_addr + ks * L::kKV + off, 16, 1024), idesc_s,
-                                            k > 0);
-                        }
-                        tc::mma_commit(&s_full[s]);
-                        tc::mma_commit(&k_empty[ks]);
-                        if (t == it.ntiles - 1) tc::mma_commit(q_empty);
-                    }
-                    __syncwarp();
-                }
-                if (t > 0) {
-                    // ---- O (+)= P_{t-1} V_{t-1}  (P from tensor memory)
-                    const int tp = t - 1;
-                    const uint32_t T = kv_iter + tp;
-                    const int s = (int)(T % kVStages);  // V stage
-                    NPV_WAIT(p_full, T & 1);
-                    NPV_WAIT(&v_full[s], (T / kVStages) & 1);
-                    if (tp == 0) NPV_WAIT(o_free, (item_iter & 1) ^ 1);
-                    const int valid = min(kTileN, it.kv_end - tp * kTileN);
+                    const int j = (int)(T & 1);
+                    const int vs = (int)(T % kVStages);
+                    NPV_WAIT(&p_full[j], (T >> 1) & 1);
+                    NPV_WAIT(&v_full[vs], (T / kVStages) & 1);
+                    if (t == 0) NPV_WAIT(o_free, (item_iter & 1) ^ 1);
+                    const int valid = min(kTileN, it.kv_end - t * kTileN);
                     const int ksteps = (valid + 15) / 16;
                     if (valid < ksteps * 16) {
                         // zero the V rows of the last K step that lie past the context
-                        uint8_t *vs = sV + s * L::kKV;
+                        uint8_t *vsm = sV + vs * L::kKV;
                         const int nrows = ksteps * 16 - valid;
                         for (int e = lane; e < nrows * 8 * kDBlocks; e += 32) {
                             const int db = e / (nrows * 8);
                             const int rr = valid + (e % (nrows * 8)) / 8;
                             const int ch = e % 8;
-                            *reinterpret_cast<uint4 *>(vs + db * kBlockBytes + rr * 128 + ch * 16) =
+                            *reinterpret_cast<uint4 *>(vsm + db * kBlockBytes + rr * 128 + ch * 16) =
                                 make_uint4(0, 0, 0, 0);
                         }
                         tc::fence_proxy_async_smem();
@@ -458,15 +484,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc::fence_after_sync();
                     if (lane == 0) {
-                        for (int k = 0; k < ksteps; ++k) {
-                            const uint32_t voff = k * 16 * 128;
-                            tc::mma_bf16_ts(tmem + kTmemO, tmem + kTmemP + k * 8,
-                                            tc::smem_desc_sw128(v_addr + s * L::kKV + voff, kBlockBytes, 1024),
-                                            idesc_o, tp > 0 || k > 0);
+                        const uint32_t d = tmem + kTmemO + j * D;
+                        const uint32_t a = tmem + j * kTileN;
+                        const uint64_t vd = vdesc + (uint64_t)((vs * L::kKV) >> 4);
+#pragma unroll
+                        for (int k = 0; k < kTileN / 16; ++k)
+                            if (k < ksteps) tc::mma_bf16_ts(d, a + k * 8, vd + (uint64_t)(k * 128), idesc_o, t >= 2 || k > 0);
+                        tc::mma_commit(&v_empty[vs]);
+                        if (t == it.ntiles - 1) tc::mma_commit(o_full);
+                    }
+                    __syncwarp();
+                }
+                const int ts = t + 2;
+                if (ts < it.ntiles) {
+                    // ---- S_ts = Q K_ts^T into buffer T & 1
+                    const uint32_t T = kv_iter + ts;
+                    const int ks = (int)(T % kKStages);
+                    NPV_WAIT(&k_full[ks], (T / kKStages) & 1);
+                    tc::fence_after_sync();
+                    if (lane == 0) {
+                        const uint32_t d = tmem + (T & 1) * kTileN;
+                        const uint64_t kd = kdesc + (uint64_t)((ks * L::kKV) >> 4);
+#pragma unroll
+                        for (int k = 0; k < D / 16; ++k) {
+                            const uint64_t off = (uint64_t)(((k >> 2) * kBlockBytes + (k & 3) * 32) >> 4);
+                            tc::mma_bf16_ss(d, qdesc + off, kd + off, idesc_s, k > 0);
                         }
-                        tc::mma_commit(&v_empty[s]);
-                        tc::mma_commit(p_empty);
-                        if (tp == it.ntiles - 1) tc::mma_commit(o_full);
+                        tc::mma_commit(&s_full[T & 1]);
+                        tc::mma_commit(&k_empty[ks]);
+                        if (ts == it.ntiles - 1) tc::mma_commit(q_empty);
                     }
                     __syncwarp();
                 }
@@ -474,169 +520,154 @@ __global__ void __launch_bounds__(kThreads, 1)
             kv_iter += it.ntiles;
             ++item_iter;
         }
-    } else {
-        // ======== softmax: warpgroup wg (warps 4 wg .. 4 wg + 3) owns key columns [64 wg, 64 wg + 64) ========
-        const int wg = warp >> 2;
-        const int row = (warp & 3) * 32 + lane;
+    } else if (warp >= kFirstSoftmaxWarp) {
+        // ==== softmax: warpgroup j (warps 4 + 4 j .. 7 + 4 j) takes the KV tiles T with T % 2 == j ====
+        // Registers: the launch gives every thread 168; the first warpgroup (MMA,
+        // producers) drops to 56 so that a softmax thread can hold a whole
+        // 128-key S row: 128 x 56 + 256 x 224 = 384 x 168.
+        setmaxnreg_inc224();
+        const int j = (warp - kFirstSoftmaxWarp) >> 2;
+        const int row = (warp & 3) * 32 + lane;  // warp % 4 selects the TMEM lane quarter
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const int kc0 = wg * kHalf;    // first key column of this warpgroup
-        const int oc0 = wg * (D / 2);  // first O column (and first Q element) of this warpgroup
+        const uint32_t s_cols = tmem + lane_off + j * kTileN;  // S_j, then P_j over its first 64 columns
+        const uint32_t o_cols = tmem + lane_off + kTmemO;      // O_0 at +0, O_1 at +D
+        const float sl2 = p.scale_log2;
         uint32_t kv_iter = 0, item_iter = 0;
         for (long long r = 0; r < rounds; ++r) {
             const long long idx = item_index(r);
-            if (idx >= n_items) continue;
+            if (idx >= n_items) break;
             const Item it = load_item<G>(p, idx);
             const int pos = row / G, jh = row % G;
             const bool valid_row = pos < it.npos;
-            const int lim = valid_row ? (it.L - it.n + it.p0 + pos) : (it.L - 1);
             const int lim_min = it.L - it.n + it.p0;  // smallest limit among the tile's rows
-            {
-                // ---- Q row -> tensor memory: this warpgroup's half of the row's D elements
-                uint32_t qw[D / 4];
-                if (valid_row) {
-                    const uint16_t *qrow =
-                        p.q + ((int64_t)(it.row0 + it.p0 + pos) * p.num_q_heads + it.h * G + jh) * D + oc0;
-#pragma unroll
-                    for (int v = 0; v < D / 16; ++v) {
-                        const uint4 x = ld_nc_v4(qrow + v * 8);
-                        qw[v * 4 + 0] = x.x;
-                        qw[v * 4 + 1] = x.y;
-                        qw[v * 4 + 2] = x.z;
-                        qw[v * 4 + 3] = x.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int v = 0; v < D / 4; ++v) qw[v] = 0u;
-                }
-                NPV_WAIT(q_empty, (item_iter & 1) ^ 1);  // the previous item's S products are done
-                tc::fence_after_sync();
-                if constexpr (D == 128) {
-                    tc::tmem_st32(tmem + lane_off + kTmemQ + wg * 32, qw);
-                } else {
-                    tc::tmem_st16(tmem + lane_off + kTmemQ + wg * 16, qw);
-                }
-                tc::tmem_wait_st();
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(q_full);
-            }
+            // rows past the tile's positions attend like its first row (their output is dropped)
+            const int lim = valid_row ? (lim_min + pos) : lim_min;
+            const int t_first = (int)((j - (int)(kv_iter & 1)) & 1);  // first tile of this warpgroup
             float m = -INFINITY, l = 0.f;
-            for (int t = 0; t < it.ntiles; ++t) {
+            for (int t = t_first; t < it.ntiles; t += 2) {
                 const uint32_t T = kv_iter + t;
-                const int sb = T & 1;
-                NPV_WAIT(&s_full[sb], (T >> 1) & 1);
+                NPV_WAIT(&s_full[j], (T >> 1) & 1);
                 tc::fence_after_sync();
-                float sv[kHalf];
+                float sv[kTileN];
                 {
-                    uint32_t raw[kHalf / 32][32];
+                    uint32_t raw[kTileN / 32][32];
 #pragma unroll
-                    for (int c = 0; c < kHalf / 32; ++c)
-                        tc::tmem_ld32(tmem + lane_off + sb * kTileN + kc0 + c * 32, raw[c]);
+                    for (int c = 0; c < kTileN / 32; ++c) tc::tmem_ld32(s_cols + c * 32, raw[c]);
                     tc::tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < kHalf / 32; ++c)
+                    for (int c = 0; c < kTileN / 32; ++c)
 #pragma unroll
                         for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(raw[c][e]);
                 }
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s_free[sb]);
-                const int kv0 = t * kTileN + kc0;
-                if (kv0 + kHalf - 1 > lim_min) {
+                const int kv0 = t * kTileN;
+                if (kv0 + kTileN - 1 > lim_min) {
 #pragma unroll
-                    for (int c = 0; c < kHalf; ++c)
+                    for (int c = 0; c < kTileN; ++c)
                         if (kv0 + c > lim) sv[c] = -INFINITY;
                 }
                 float mx8[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) mx8[e] = sv[e];
 #pragma unroll
-                for (int c = 8; c < kHalf; c += 8)
+                for (int c = 8; c < kTileN; c += 8)
 #pragma unroll
                     for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], sv[c + e]);
-                const float pmax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-                // full-row max: swap partial maxima with the other warpgroup
-                xmax[(sb * 2 + wg) * kTileM + row] = pmax;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&x_full[sb]);
-                NPV_WAIT(&x_full[sb], (T >> 1) & 1);
-                const float omax = xmax[(sb * 2 + (1 - wg)) * kTileM + row];
-                const float m_tile = fmaxf(pmax, omax) * p.scale_log2;
-                if (t == 0) {
+                const float m_tile = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                           fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
+                                     sl2;
+                // lazy rescale: the running max moves only when it grows by more than
+                // 2^kRescaleThreshold; O_j is then rescaled after P is written
+                float alpha = 1.0f;
+                bool rescale = false;
+                if (t == t_first) {
                     m = m_tile;
                 } else {
                     const float m_new = fmaxf(m, m_tile);
-                    const bool need = m_new > m + kRescaleThreshold;  // the same in both warpgroups
-                    if (__any_sync(0xffffffffu, need)) {
-                        // the previous P.V must have landed before O is rescaled
-                        NPV_WAIT(p_empty, (T - 1) & 1);
-                        tc::fence_after_sync();
-                        const float alpha = need ? fast_exp2(m - m_new) : 1.0f;
-                        // this warpgroup's half of O, 32 columns at a time
-#pragma unroll
-                        for (int c = 0; c < D / 64; ++c) {
-                            uint32_t raw[32];
-                            const uint32_t ta = tmem + lane_off + kTmemO + oc0 + c * 32;
-                            tc::tmem_ld32(ta, raw);
-                            tc::tmem_wait_ld();
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
-                            tc::tmem_st32(ta, raw);
-                        }
-                        tc::tmem_wait_st();
-                        if (need) {
-                            l *= alpha;
-                            m = m_new;
-                        }
+                    const bool need = m_new > m + kRescaleThreshold;
+                    rescale = __any_sync(0xffffffffu, need);
+                    if (need) {
+                        alpha = fast_exp2(m - m_new);
+                        l *= alpha;
+                        m = m_new;
                     }
                 }
-                // probabilities of this warpgroup's 64 keys, packed to bf16 pairs, into P's
-                // columns [32 wg, 32 wg + 32) of tensor memory
+                // a row with every key so far masked keeps m = -inf: its probabilities are 0
+                const float m_use = (m == -INFINITY) ? 0.f : m;
                 float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                uint32_t pk[kHalf / 2];
 #pragma unroll
-                for (int c = 0; c < kHalf; c += 2) {
-                    const float p0v = fast_exp2(fmaf(sv[c], p.scale_log2, -m));
-                    const float p1v = fast_exp2(fmaf(sv[c + 1], p.scale_log2, -m));
-                    ls8[(c / 2) & 7] += p0v + p1v;
-                    pk[c / 2] = pack_bf16x2(p0v, p1v);
+                for (int c = 0; c < kTileN; ++c) {
+                    sv[c] = fast_exp2(fmaf(sv[c], sl2, -m_use));  // in place: S -> P
+                    ls8[c & 7] += sv[c];
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(sv[h * 64 + 2 * c], sv[h * 64 + 2 * c + 1]);
+                    tc::tmem_st32(s_cols + h * 32, pk);
                 }
                 l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
-                if (T > 0) NPV_WAIT(p_empty, (T - 1) & 1);  // the previous P.V has read P
-                tc::fence_after_sync();
-                tc::tmem_st32(tmem + lane_off + kTmemP + wg * (kHalf / 2), pk);
+                if (rescale) {
+                    // O_j: its last P.V finished before S_t (issued after it) completed,
+                    // and the next one waits for p_full below
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t raw[32];
+                        const uint32_t ta = o_cols + j * D + c * 32;
+                        tc::tmem_ld32(ta, raw);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
+                        tc::tmem_st32(ta, raw);
+                    }
+                }
                 tc::tmem_wait_st();
                 tc::fence_before_sync();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(p_full);
+                if (lane == 0) mbar_arrive(&p_full[j]);
             }
-            // ---- epilogue: full row sum from the two partial sums, then O / l -> bf16
-            xsum[wg * kTileM + row] = l;
+            // ---- epilogue: merge the two warpgroups' partial results, O / l -> bf16
+            // (double-buffered by item parity: the other warpgroup may still read
+            // this item's slot when this one reaches the next item's epilogue)
+            float2 *xml_item = xml + (item_iter & 1) * 2 * kTileM;
+            xml_item[j * kTileM + row] = make_float2(m, l);
             __syncwarp();
-            if (lane == 0) mbar_arrive(l_full);
-            NPV_WAIT(l_full, item_iter & 1);
+            if (lane == 0) mbar_arrive(ml_full);
+            NPV_WAIT(ml_full, item_iter & 1);
             NPV_WAIT(o_full, item_iter & 1);
             tc::fence_after_sync();
             {
-                const float lo = xsum[(1 - wg) * kTileM + row];
-                uint32_t raw[D / 64][32];
+                const float2 mo = xml_item[(1 - j) * kTileM + row];
+                const bool has_me = t_first < it.ntiles, has_other = (1 - t_first) < it.ntiles;
+                float mm = fmaxf(has_me ? m : -INFINITY, has_other ? mo.x : -INFINITY);
+                const float a_me = has_me ? fast_exp2(m - mm) : 0.f;
+                const float a_ot = has_other ? fast_exp2(mo.x - mm) : 0.f;
+                const float inv = 1.0f / (a_me * l + a_ot * mo.y);
+                const float a0 = j == 0 ? a_me : a_ot, a1 = j == 0 ? a_ot : a_me;
+                const bool has0 = j == 0 ? has_me : has_other, has1 = j == 0 ? has_other : has_me;
+                // this warpgroup writes output columns [j D / 2, (j + 1) D / 2)
+                uint16_t *orow = p.out + ((int64_t)(it.row0 + it.p0 + pos) * p.num_q_heads + it.h * G + jh) * D +
+                                 j * (D / 2);
 #pragma unroll
-                for (int c = 0; c < D / 64; ++c) tc::tmem_ld32(tmem + lane_off + kTmemO + oc0 + c * 32, raw[c]);
-                tc::tmem_wait_ld();
-                const float inv = 1.0f / (l + lo);
-                uint16_t *orow =
-                    p.out + ((int64_t)(it.row0 + it.p0 + pos) * p.num_q_heads + it.h * G + jh) * D + oc0;
-                if (valid_row) {
-#pragma unroll
-                    for (int c = 0; c < D / 64; ++c)
+                for (int c = 0; c < D / 64; ++c) {
+                    uint32_t r0[32], r1[32];
+                    const uint32_t col = j * (D / 2) + c * 32;
+                    if (has0) tc::tmem_ld32(o_cols + col, r0);
+                    if (has1) tc::tmem_ld32(o_cols + D + col, r1);
+                    tc::tmem_wait_ld();
+                    if (valid_row) {
 #pragma unroll
                         for (int v = 0; v < 4; ++v) {
                             float f[8];
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(raw[c][v * 8 + e]) * inv;
+                            for (int e = 0; e < 8; ++e) {
+                                const float x0 = has0 ? __uint_as_float(r0[v * 8 + e]) * a0 : 0.f;
+                                const float x1 = has1 ? __uint_as_float(r1[v * 8 + e]) * a1 : 0.f;
+                                f[e] = (x0 + x1) * inv;
+                            }
                             st_global_v4(orow + c * 32 + v * 8, pack8(f));
                         }
+                    }
                 }
             }
             tc::fence_before_sync();
