@@ -32,7 +32,7 @@
 //     exponential phases interleave on the special-function units.
 //   * Warp roles: warp 0 owns tensor memory and issues tcgen05.mma from one
 //     thread; warp 1 issues the TMA loads of the K tiles (128 keys) through a
-//     3-stage ring, warp 2 those of the V tiles through a 2-stage ring (block ids
+//     3-stage ring, warp 2 those of the V tiles through a 3-stage ring (block ids
 //     from the block table a 32-entry window at a time, one TMA box per block
 //     piece); warp 3 loads each item's Q tile with one TMA box per 64 columns.
 //     The first warpgroup gives registers to the softmax warpgroups (setmaxnreg)
@@ -59,7 +59,7 @@ namespace prefill {
 constexpr int kTileM = 128;   // query rows per item (MMA M)
 constexpr int kTileN = 128;   // keys per KV tile (MMA N of S, K of P.V)
 constexpr int kKStages = 3;   // K ring depth (a K stage is free once S = Q K^T is done)
-constexpr int kVStages = 2;   // V ring depth (a V stage is free once O += P V is done)
+constexpr int kVStages = 3;   // V ring depth (a V stage is free once O += P V is done)
 constexpr int kThreads = 384;  // MMA, K producer, V producer, Q producer, 8 softmax warps
 constexpr int kMmaWarp = 0;
 constexpr int kKProducerWarp = 1;
@@ -90,14 +90,16 @@ struct Params {
     int32_t *plan_count;  // [1]: number of (sequence, row-tile) pairs
     int2 *plan_pairs;     // [max_pairs]: (sequence, row tile), longest first
     int32_t max_pairs;
+    float2 *ml_x;         // [grid][2 item parities][2 warpgroups][128 rows]: (m, l) exchange
 };
 
-// Shared-memory layout (bytes from a 1024-aligned base): barriers and the
-// warpgroups' (m, l) exchange, then the Q tile and the K and V rings.
+// Shared-memory layout (bytes from a 1024-aligned base): barriers, then the Q
+// tile and the K and V rings (3 + 3 stages of 32 KB at D = 128: 225 KB in all,
+// which is why the warpgroups' per-item (m, l) exchange goes through a
+// CTA-private slot in global memory instead).
 template <int D>
 struct Smem {
-    static constexpr int kHeader = 5120;
-    static constexpr int kXml = 1024;  // float2 [2 item parities][2 warpgroups][128 rows]
+    static constexpr int kHeader = 1024;
     static constexpr int kKV = kTileN * D * 2;
     static constexpr int q = kHeader;
     static constexpr int k = q + kTileM * D * 2;
@@ -333,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *ml_full = o_free + 1;         // per-row (m, l) of both warpgroups exchanged (8 softmax warps)
     uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(ml_full + 1);
     int *abort_flag = reinterpret_cast<int *>(ml_full + 2);
-    float2 *xml = reinterpret_cast<float2 *>(smem + L::kXml);  // [2 item parities][2 warpgroups][128 rows]
+    float2 *xml = p.ml_x + (size_t)blockIdx.x * (2 * 2 * kTileM);  // this CTA's exchange slots
     uint8_t *sQ = smem + L::q;
     uint8_t *sK = smem + L::k;
     uint8_t *sV = smem + L::v;
@@ -628,7 +630,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // ---- epilogue: merge the two warpgroups' partial results, O / l -> bf16
             // (double-buffered by item parity: the other warpgroup may still read
-            // this item's slot when this one reaches the next item's epilogue)
+            // this item's slot when this one reaches the next item's epilogue; the
+            // mbarrier's release / acquire orders these global accesses in the CTA)
             float2 *xml_item = xml + (item_iter & 1) * 2 * kTileM;
             xml_item[j * kTileM + row] = make_float2(m, l);
             __syncwarp();
