@@ -39,6 +39,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "paged GQA decode attention: achieved HBM GB/s (% of peak), tokens/s"
 MIXED_METRIC = "chunked-prefill mixed batch attention: HBM GB/s, tokens/s, prefill TFLOP/s"
+SPEC_METRIC = "speculative-decode verify attention (multi-row decode over the paged cache): HBM GB/s, tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 KERNEL_SRC = os.path.join(ROOT, "paged_kv_cache_bf16_b200", "csrc", "decode_attention.cuh")
@@ -156,11 +157,27 @@ def whole_job_rate(ranks: Ranks, local_units: float, local_ms: float) -> tuple:
 # workload bookkeeping (host side)
 # ---------------------------------------------------------------------------
 
-def step_bytes(wl, step, seqs=None):
+def kv_tokens(wl, step, seqs):
+    """(logical, unique) K/V token rows the attention of `seqs` reads: a physical block
+    shared by several sequences counts once in `unique`, for the most tokens any of
+    them reads from it."""
+    L = wl.context_lens(step).astype(np.int64)
+    logical = int(L[seqs].sum())
+    used = {}
+    for b in seqs:
+        nblk = -(-int(L[b]) // wl.BS)
+        for i, blk in enumerate(wl.seq_blocks[b][:nblk]):
+            n = min(wl.BS, int(L[b]) - i * wl.BS)
+            used[int(blk)] = max(used.get(int(blk), 0), n)
+    return logical, int(sum(used.values()))
+
+
+def step_bytes(wl, step, seqs=None, logical=False):
     """Algorithmic HBM bytes of one step over `seqs` (default all): (store, attention).
 
-    Attention reads each sequence's live K/V once, reads q, writes out and reads
-    the metadata; the store reads and writes each new K/V row once."""
+    Attention reads each live K/V row once (a block shared by several sequences
+    once, unless `logical`), reads q, writes out and reads the metadata; the store
+    reads and writes each new K/V row once."""
     seqs = np.arange(wl.B) if seqs is None else np.asarray(seqs)
     row = wl.Hkv * wl.D * 2
     nq = int(wl.query_lens[seqs].sum())
@@ -168,7 +185,8 @@ def step_bytes(wl, step, seqs=None):
     L = wl.context_lens(step).astype(np.int64)[seqs]
     qo = 2 * nq * wl.Hq * wl.D * 2
     meta = len(seqs) * 8 + int(sum(-(-int(x) // wl.BS) for x in L)) * 4
-    attn = int(L.sum()) * 2 * row + qo + meta
+    n_log, n_uni = kv_tokens(wl, step, seqs)
+    attn = (n_log if logical else n_uni) * 2 * row + qo + meta
     return store, attn
 
 
@@ -399,9 +417,11 @@ def npv_arm(args, rank, world, local_rank):
     barrier = ranks.barrier
     max_over_ranks = ranks.max
 
-    bytes_steps = [step_bytes(wl, i % nsteps) for i in range(args.steps)]
+    per_step = [step_bytes(wl, i) for i in range(nsteps)]
+    bytes_steps = [per_step[i % nsteps] for i in range(args.steps)]
     store_bytes = sum(b[0] for b in bytes_steps)
     attn_bytes = sum(b[1] for b in bytes_steps)
+    logical_attn = sum(step_bytes(wl, i, logical=True)[1] for i in range(nsteps)) / nsteps
 
     for i in range(args.warmup):
         step(i)
@@ -474,7 +494,9 @@ def npv_arm(args, rank, world, local_rank):
     launch_ms = (ms / args.steps) if not (mixed or args.separate_store) else call_ms
     achieved = call_bytes / (launch_ms * 1e-3) / 1e9
     line = {
-        "metric": METRIC if not mixed else MIXED_METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "metric": (METRIC if not mixed else
+                   SPEC_METRIC if wl.spec.prefill_seqs == wl.B and wl.spec.prefill_len <= 8 else MIXED_METRIC),
+        "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(wl),
@@ -483,6 +505,10 @@ def npv_arm(args, rank, world, local_rank):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
+    if wl.spec.share_group:
+        # prefix-shared blocks: the GB/s above count each shared block once
+        line["kv_bytes_per_step"] = {"unique": attn_bytes / args.steps, "logical": logical_attn}
+        line["logical_gb_s"] = ranks.sum((logical_attn + store_bytes / args.steps) * args.steps) / (ms * 1e-3) / 1e9
     if not mixed:
         line["roofline"] = {
             "kernel": ("npv_paged_decode_attention" if args.separate_store else
@@ -520,6 +546,8 @@ def mixed_subbatches(args, wl, st, dev, stream, ops, W, timed):
     res = {}
     for kind in ("prefill", "decode"):
         seqs = [b for b in range(wl.B) if (wl.query_lens[b] > 1) == (kind == "prefill")]
+        if not seqs:
+            continue
         rows = np.concatenate([np.arange(cu[b], cu[b + 1]) for b in seqs])
         ridx = torch.from_numpy(rows).to(dev)
         bidx = torch.from_numpy(np.array(seqs)).to(dev)
@@ -545,13 +573,23 @@ def mixed_subbatches(args, wl, st, dev, stream, ops, W, timed):
         res[kind] = {"ms": ms, "gb_s": nbytes / (ms * 1e-3) / 1e9, "tflop_s": fl / (ms * 1e-3) / 1e12,
                      "rows": int(cus[-1]), "seqs": len(seqs)}
     pre = res["prefill"]
-    roof = {"kernel": "npv_paged_prefill_attention on the 16 prefill sequences (plan + tcgen05 kernel)",
-            "bound": "tensor", "achieved": pre["tflop_s"], "peak": tflops_peak, "unit": "TFLOP/s",
-            "frac": pre["tflop_s"] / tflops_peak, "peak_source": tf_kind, "traffic": None,
-            "algorithmic_flops_per_launch": prefill_flops(wl, 0, [b for b in range(wl.B) if wl.query_lens[b] > 1]),
-            "mean_launch_ms": pre["ms"]}
-    return {"roofline": roof, "prefill_part": pre,
-            "decode_part": dict(res["decode"], pct_of_peak_hbm=100 * res["decode"]["gb_s"] / hbm_peak)}
+    pre_seqs = [b for b in range(wl.B) if wl.query_lens[b] > 1]
+    name = f"npv_paged_prefill_attention on the {len(pre_seqs)} multi-row sequences (plan + tcgen05 kernel)"
+    # the binding resource of the multi-row part: tensor pipe (long chunks) or HBM
+    # (a few rows per sequence, e.g. speculative-decode verification)
+    if pre["tflop_s"] / tflops_peak >= pre["gb_s"] / hbm_peak:
+        roof = {"kernel": name, "bound": "tensor", "achieved": pre["tflop_s"], "peak": tflops_peak,
+                "unit": "TFLOP/s", "frac": pre["tflop_s"] / tflops_peak, "peak_source": tf_kind, "traffic": None,
+                "algorithmic_flops_per_launch": prefill_flops(wl, 0, pre_seqs), "mean_launch_ms": pre["ms"]}
+    else:
+        roof = {"kernel": name, "bound": "hbm", "achieved": pre["gb_s"], "peak": hbm_peak, "unit": "GB/s",
+                "frac": pre["gb_s"] / hbm_peak, "peak_source": "measured: MEASURED_PEAKS.json hbm_gbs",
+                "traffic": None, "algorithmic_bytes_per_launch": step_bytes(wl, 0, pre_seqs)[1],
+                "mean_launch_ms": pre["ms"]}
+    out = {"roofline": roof, "prefill_part": pre}
+    if "decode" in res:
+        out["decode_part"] = dict(res["decode"], pct_of_peak_hbm=100 * res["decode"]["gb_s"] / hbm_peak)
+    return out
 
 
 def npv_e2e(args, wl, st, ws, dev, stream, ops, W, barrier, max_over_ranks, kind):

@@ -393,7 +393,7 @@ def draw(spec: Spec) -> Workload:
                     max_blocks_per_seq=mb)
 
 
-# The five named workloads.  `seed` is the workload's index.
+# The named workloads.  `seed` is the workload's index.
 SPECS: Dict[str, Spec] = {
     "tiny_decode": Spec(
         name="tiny_decode", seed=1, num_seqs=4, num_q_heads=4, num_kv_heads=2, head_dim=64,
@@ -415,6 +415,11 @@ SPECS: Dict[str, Spec] = {
         block_size=256, num_blocks=57344, sigma=0.5, ctx_lo=32768, ctx_hi=131072,
         description="long-context split-KV decode: 8 seqs, L~U[32768,131072], 32 Q / 8 KV heads, "
                     "D=128, BS=256, N(0,0.5^2); 57,344-block (~60 GB) pool"),
+    "spec_verify_decode": Spec(
+        name="spec_verify_decode", seed=6, num_seqs=256, num_q_heads=16, num_kv_heads=8, head_dim=128,
+        block_size=256, num_blocks=4096, prefill_seqs=256, prefill_len=4, prior_lo=100, prior_hi=2044,
+        description="speculative-decode verification: 256 seqs x 4 query rows (3 draft tokens + 1) "
+                    "over prior context U[100,2044]; 16 Q / 8 KV heads, D=128, BS=256"),
     "chunked_prefill_mixed": Spec(
         name="chunked_prefill_mixed", seed=5, num_seqs=256, num_q_heads=16, num_kv_heads=8, head_dim=128,
         block_size=256, num_blocks=4096, ctx_lo=100, ctx_hi=2048, prefill_seqs=16, prefill_len=512,

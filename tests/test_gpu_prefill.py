@@ -120,6 +120,18 @@ def test_prefill_mixed_named_workload_sampled():
     assert_close(out[torch.from_numpy(rows).to(DEV)], ref, "prefill rows")
 
 
+def test_prefill_spec_verify_named_workload():
+    """Speculative-decode verification: 256 sequences x 4 query rows over priors up to 2,044,
+    every row checked against the oracle."""
+    wl = W.workload("spec_verify_decode")
+    st = W.DeviceState(wl, DEV)
+    run_store(st, 0)
+    out = run_prefill(st)
+    no_device_errors()
+    ref, rows = oracle_compact(wl, 0)
+    assert_close(out[torch.from_numpy(rows).to(DEV)], ref, "spec verify rows")
+
+
 def test_prefill_decode_rows_equal_decode_call():
     """Rows with n_b == 1 inside a prefill call give the decode call's bits."""
     spec = tiny_spec(name="p_dec", seed=813, head_dim=128, num_q_heads=16, num_kv_heads=8, block_size=256,

@@ -51,7 +51,8 @@ def test_named_workload_metadata(name):
         assert pre.sum() == s.prefill_seqs and (wl.query_lens[pre] == s.prefill_len).all()
         prior = L[pre] - s.prefill_len
         assert prior.min() >= s.prior_lo and prior.max() <= s.prior_hi
-        assert L[~pre].min() >= s.ctx_lo and L[~pre].max() <= s.ctx_hi
+        if (~pre).any():
+            assert L[~pre].min() >= s.ctx_lo and L[~pre].max() <= s.ctx_hi
     else:
         assert L.min() >= s.ctx_lo and L.max() <= s.ctx_hi
     for step in (0, s.num_steps - 1):
