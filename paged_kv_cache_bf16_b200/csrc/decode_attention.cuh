@@ -424,10 +424,12 @@ __global__ void __launch_bounds__((max_heads_per_cta(G) + 1) * 32, 1) decode_spl
                 unpack8(ld_shared_v4(kst + (uint32_t)(i * RPL + rg) * tok_bytes), kf);
 #pragma unroll
                 for (int j = 0; j < G; ++j) {
-                    float a = qf[j][0] * kf[0];
+                    // even and odd dims accumulate in the two halves of a pair
+                    float2 a = fmul2(make_float2(qf[j][0], qf[j][1]), make_float2(kf[0], kf[1]));
 #pragma unroll
-                    for (int e = 1; e < 8; ++e) a = fmaf(qf[j][e], kf[e], a);
-                    acc[i][j] = a;
+                    for (int e = 2; e < 8; e += 2)
+                        a = ffma2(make_float2(qf[j][e], qf[j][e + 1]), make_float2(kf[e], kf[e + 1]), a);
+                    acc[i][j] = a.x + a.y;
                 }
             }
             // ---- reduce-scatter over the row's lanes: halve the token list at
@@ -498,7 +500,12 @@ __global__ void __launch_bounds__((max_heads_per_cta(G) + 1) * 32, 1) decode_spl
                     for (int j = 0; j < G; ++j) {
                         const float pv = my_p[tok * G + j];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) o[j][e] = fmaf(pv, vf[e], o[j][e]);
+                        for (int e = 0; e < 8; e += 2) {
+                            const float2 r = ffma2(make_float2(pv, pv), make_float2(vf[e], vf[e + 1]),
+                                                   make_float2(o[j][e], o[j][e + 1]));
+                            o[j][e] = r.x;
+                            o[j][e + 1] = r.y;
+                        }
                     }
                 }
             }
