@@ -196,7 +196,9 @@ NPV_API size_t npv_paged_prefill_workspace_size(int32_t num_seqs, int32_t total_
  *                 including its n_b new rows, which must already be stored.
  *                 Row i of sequence b sits at position L_b - n_b + i and sees
  *                 keys 0 .. L_b - n_b + i.  L_b < n_b sets NPV_DEVERR_CONTEXT_LEN.
- *   max_seqlen_q  host upper bound on n_b (used to size the launch).
+ *   max_seqlen_q  host upper bound on n_b, the flash-attn-style hint; checked to be
+ *                 >= 0 and otherwise unused (the plan kernel reads the row counts
+ *                 on the device).
  *   other arguments as for npv_paged_decode_attention.
  * Rows with n_b >= 2 run on the tcgen05 tensor cores (QK^T and PV with fp32
  * accumulators in tensor memory; P rounded to bf16 for the PV product); rows
