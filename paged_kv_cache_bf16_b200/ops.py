@@ -93,6 +93,25 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+def _on_one_gpu(what: str, bf16=(), other=()) -> None:
+    """Every tensor a call hands to the kernels must live on one CUDA device (a host
+    pointer would be dereferenced by the GPU); the activation and cache tensors must
+    be bf16.  Raises before anything is launched."""
+    dev = None
+    for name, t in list(bf16) + list(other):
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise ValueError(f"{what}: {name} must be a CUDA tensor")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{what}: {name} is on {t.device}, the other tensors on {dev}")
+    for name, t in bf16:
+        if t is not None and t.dtype != torch.bfloat16:
+            raise TypeError(f"{what}: {name} must be torch.bfloat16, got {t.dtype}")
+
+
 def _cache_shape(k_cache: torch.Tensor):
     assert k_cache.dim() == 4 and k_cache.is_contiguous(), "cache must be [num_blocks, block_size, Hkv, D]"
     return k_cache.shape
@@ -101,6 +120,8 @@ def _cache_shape(k_cache: torch.Tensor):
 def store_kvcache(key: torch.Tensor, value: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                   slot_mapping: torch.Tensor, stream=None) -> None:
     """Scatter key/value [T, Hkv, D] bf16 into the caches at slot_mapping [T] int32."""
+    _on_one_gpu("store_kvcache", bf16=[("key", key), ("value", value), ("k_cache", k_cache), ("v_cache", v_cache)],
+                other=[("slot_mapping", slot_mapping)])
     NB, BS, Hkv, D = _cache_shape(k_cache)
     T = slot_mapping.shape[0]
     assert slot_mapping.dtype == torch.int32
@@ -129,6 +150,9 @@ def paged_decode_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
                            out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                            stream=None) -> torch.Tensor:
     """Decode attention: q [B, Hq, D] bf16 -> out [B, Hq, D] bf16."""
+    _on_one_gpu("paged_decode_attention",
+                bf16=[("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("out", out)],
+                other=[("block_tables", block_tables), ("context_lens", context_lens), ("workspace", workspace)])
     NB, BS, Hkv, D = _cache_shape(k_cache)
     B, Hq, Dq = q.shape
     assert Dq == D and q.stride(2) == 1 and q.stride(1) == D
@@ -151,6 +175,11 @@ def store_kvcache_and_decode_attention(q: torch.Tensor, key: torch.Tensor, value
                                        workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """One decode step in one launch set: store key/value [B, Hkv, D] at slot_mapping [B], then
     decode attention for q [B, Hq, D] -> out [B, Hq, D]."""
+    _on_one_gpu("store_kvcache_and_decode_attention",
+                bf16=[("q", q), ("key", key), ("value", value), ("k_cache", k_cache), ("v_cache", v_cache),
+                      ("out", out)],
+                other=[("slot_mapping", slot_mapping), ("block_tables", block_tables), ("context_lens", context_lens),
+                       ("workspace", workspace)])
     NB, BS, Hkv, D = _cache_shape(k_cache)
     B, Hq, Dq = q.shape
     assert Dq == D and q.stride(2) == 1 and q.stride(1) == D
@@ -175,6 +204,10 @@ def paged_prefill_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: tor
                             out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                             stream=None) -> torch.Tensor:
     """Varlen causal attention: q [total_q, Hq, D] packed by cu_seqlens_q -> out [total_q, Hq, D]."""
+    _on_one_gpu("paged_prefill_attention",
+                bf16=[("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("out", out)],
+                other=[("cu_seqlens_q", cu_seqlens_q), ("block_tables", block_tables), ("context_lens", context_lens),
+                       ("workspace", workspace)])
     NB, BS, Hkv, D = _cache_shape(k_cache)
     total_q, Hq, Dq = q.shape
     B = context_lens.shape[0]
