@@ -43,6 +43,7 @@ SPEC_METRIC = "speculative-decode verify attention (multi-row decode over the pa
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 KERNEL_SRC = os.path.join(ROOT, "paged_kv_cache_bf16_b200", "csrc", "decode_attention.cuh")
+PREFILL_SRC = os.path.join(ROOT, "paged_kv_cache_bf16_b200", "csrc", "prefill_attention.cuh")
 
 
 def parse_args(argv=None):
@@ -83,15 +84,16 @@ def measured_tflops():
         return 1590.0, "fallback 1590 TFLOP/s"
 
 
-def kernel_source_hash() -> str:
-    with open(KERNEL_SRC, "rb") as f:
+def kernel_source_hash(src: str = None) -> str:
+    with open(src or KERNEL_SRC, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per launch of the split kernel from the committed ncu summary,
-    or None if there is none or the kernel source changed since the capture."""
-    path = os.path.join(PROFILE_DIR, f"decode_split_{workload}.txt")
+def profiled_traffic(workload: str, kernel: str = "decode_split", src: str = None):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary
+    profiles/<kernel>_<workload>.txt, or None if there is none or the kernel's
+    source (`src`, default the decode kernel's) changed since the capture."""
+    path = os.path.join(PROFILE_DIR, f"{kernel}_{workload}.txt")
     try:
         text = open(path).read()
     except OSError:
@@ -101,7 +103,7 @@ def profiled_traffic(workload: str):
         if ":" in line:
             k, v = line.split(":", 1)
             vals[k.strip()] = v.strip()
-    if vals.get("kernel_source_sha256_16") != kernel_source_hash():
+    if vals.get("kernel_source_sha256_16") != kernel_source_hash(src):
         return None
     try:
         return float(vals["dram_bytes_per_launch_full_workload"])
@@ -603,8 +605,10 @@ def mixed_subbatches(args, wl, st, dev, stream, ops, W, timed):
     # the binding resource of the multi-row part: tensor pipe (long chunks) or HBM
     # (a few rows per sequence, e.g. speculative-decode verification)
     if pre["tflop_s"] / tflops_peak >= pre["gb_s"] / hbm_peak:
+        traffic = profiled_traffic(wl.spec.name, "prefill_attention", PREFILL_SRC)
         roof = {"kernel": name, "bound": "tensor", "achieved": pre["tflop_s"], "peak": tflops_peak,
-                "unit": "TFLOP/s", "frac": pre["tflop_s"] / tflops_peak, "peak_source": tf_kind, "traffic": None,
+                "unit": "TFLOP/s", "frac": pre["tflop_s"] / tflops_peak, "peak_source": tf_kind,
+                "traffic": traffic,
                 "algorithmic_flops_per_launch": prefill_flops(wl, 0, pre_seqs), "mean_launch_ms": pre["ms"]}
     else:
         roof = {"kernel": name, "bound": "hbm", "achieved": pre["gb_s"], "peak": hbm_peak, "unit": "GB/s",
