@@ -84,6 +84,15 @@ def measured_tflops():
         return 1590.0, "fallback 1590 TFLOP/s"
 
 
+def metric_for(wl) -> str:
+    """The metric string of a workload's JSON line (the same for both arms)."""
+    if wl.spec.prefill_seqs == 0:
+        return METRIC
+    if wl.spec.prefill_seqs == wl.B and wl.spec.prefill_len <= 8:
+        return SPEC_METRIC
+    return MIXED_METRIC
+
+
 def kernel_source_hash(src: str = None) -> str:
     with open(src or KERNEL_SRC, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
@@ -350,7 +359,7 @@ def reference_arm(args, rank, world):
     value = nbytes / dt / 1e9
     sample = (f"each step: the fp64 C oracle's store + decode attention for {n} of the {wl.B} sequences of "
               f"{wl.spec.name} ({runner.threads} threads)")
-    line = {"metric": METRIC, "value": value, "unit": "GB/s", "impl": "reference", "n_gpus": args.gpus,
+    line = {"metric": metric_for(wl), "value": value, "unit": "GB/s", "impl": "reference", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(wl),
@@ -519,8 +528,7 @@ def npv_arm(args, rank, world, local_rank):
     launch_ms = (ms / args.steps) if not (mixed or args.separate_store) else call_ms
     achieved = call_bytes / (launch_ms * 1e-3) / 1e9
     line = {
-        "metric": (METRIC if not mixed else
-                   SPEC_METRIC if wl.spec.prefill_seqs == wl.B and wl.spec.prefill_len <= 8 else MIXED_METRIC),
+        "metric": metric_for(wl),
         "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
