@@ -42,7 +42,9 @@
  * 1 / sqrt(head_dim) (same section, step 2).
  *
  * Supported: head_dim in {64, 128}; num_q_heads / num_kv_heads in {1, 2, 4, 8};
- * block_size a positive multiple of 16; every bf16 pointer 16-byte aligned.
+ * block_size a positive multiple of 16; every bf16 pointer 16-byte aligned;
+ * for npv_paged_prefill_attention, num_blocks * block_size < 2^31 (its tensor
+ * maps address cache rows with signed 32-bit coordinates).
  */
 #ifndef NPV_H
 #define NPV_H

@@ -452,7 +452,8 @@ npv_status npv_paged_prefill_attention(void *out, const void *q, const int32_t *
     if (num_q_heads <= 0 || num_q_heads % num_kv_heads != 0) return NPV_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return NPV_ERR_INVALID_ARG;
     if (block_size % 16 != 0) return NPV_ERR_UNSUPPORTED;
-    if ((int64_t)num_blocks * block_size > 0xFFFFFFFFll) return NPV_ERR_UNSUPPORTED;
+    // TMA coordinates are signed 32-bit: every cache slot row must be addressable
+    if ((int64_t)num_blocks * block_size > 0x7FFFFFFFll) return NPV_ERR_UNSUPPORTED;
     PrefillConfig cfg;
     npv_status st = prefill_config(num_seqs, total_q, num_q_heads, num_kv_heads, head_dim, &cfg);
     if (st != NPV_OK) return st;
