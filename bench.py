@@ -59,6 +59,8 @@ def parse_args(argv=None):
                     help="decode steps as npv_store_kvcache + npv_paged_decode_attention instead of the fused call")
     ap.add_argument("--graph", action="store_true",
                     help="time the fused decode steps replayed from one CUDA graph of the workload's step cycle")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the other workloads' block in the headline line")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline budget")
     ap.add_argument("--ref-seconds", type=float, default=150.0, help="reference-arm budget")
     return ap.parse_args(argv)
@@ -499,7 +501,7 @@ def npv_arm(args, rank, world, local_rank):
 
     extra = {}
     if mixed:
-        extra = mixed_subbatches(args, wl, st, dev, stream, ops, W, timed)
+        extra = mixed_subbatches(args.steps, wl, st, dev, stream, ops, W, timed)
 
     # keep the GPU loaded long enough for the clock sampler to see it
     t_end = time.time() + 1.5
@@ -552,6 +554,8 @@ def npv_arm(args, rank, world, local_rank):
             "peak_source": f"{peak_kind}: MEASURED_PEAKS.json hbm_gbs" if peak_kind == "measured"
             else "fallback 6650 GB/s",
             "traffic": profiled_traffic(args.workload) if not args.separate_store else None,
+            "traffic_source": (f"copied from the ncu capture in profiles/decode_split_{args.workload}.txt "
+                               "(kept only while the kernel source hash matches the capture's)"),
             "algorithmic_bytes_per_launch": call_bytes, "mean_launch_ms": launch_ms,
             "isolated_call_ms": call_ms}
     else:
@@ -559,6 +563,10 @@ def npv_arm(args, rank, world, local_rank):
         line.update(extra)
     if e2e is not None:
         line["e2e"] = e2e
+    if world == 1 and not args.no_secondary and args.workload == W.HEADLINE and not args.graph:
+        del st, ws, out
+        torch.cuda.empty_cache()
+        line["secondary"] = secondary(args, dev, stream, ops, W, timed)
     if rank == 0 and not args.no_cpu_baseline and not mixed:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
     if rank == 0:
@@ -566,11 +574,69 @@ def npv_arm(args, rank, world, local_rank):
     return 0
 
 
+# The other named workloads, measured in the headline run (one GPU) so that each
+# has a record beside the headline: GQA 4:1 decode with prefix-shared blocks,
+# long-context split-KV decode, the chunked-prefill mix and speculative-decode
+# verification.
+SECONDARY = ("llama8b_prefix_decode", "long_context_decode", "chunked_prefill_mixed", "spec_verify_decode")
+
+
+def secondary(args, dev, stream, ops, W, timed):
+    """One short timed loop per secondary workload (inputs resident; CUDA events)."""
+    import torch
+
+    hbm_peak, _ = measured_peaks()
+    steps = max(3, min(args.steps, 30))
+    res = {"steps": steps, "warmup": 3,
+           "note": "each workload's own step (decode: fused store + decode call; mixed and verify: store + "
+                   "prefill call), timed like the headline; bytes as the headline counts them"}
+    for name in SECONDARY:
+        wl = W.workload(name)
+        st = W.DeviceState(wl, dev)
+        s = st.steps[0]
+        mixed = wl.spec.prefill_seqs > 0
+        if mixed:
+            ws = ops.alloc_workspace(ops.prefill_workspace_size(wl.B, wl.total_q, wl.Hq, wl.Hkv, wl.D), dev)
+        else:
+            ws = ops.alloc_workspace(ops.decode_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.D), dev)
+        out = torch.empty((wl.total_q, wl.Hq, wl.D), dtype=torch.bfloat16, device=dev)
+
+        def step(i):
+            if mixed:
+                ops.store_kvcache(s["key"], s["value"], st.k_cache, st.v_cache, s["slot_mapping"])
+                ops.paged_prefill_attention(s["q"], st.k_cache, st.v_cache, s["cu_seqlens_q"], s["max_seqlen_q"],
+                                            s["block_tables"], s["context_lens"], out=out, workspace=ws)
+            else:
+                ops.store_kvcache_and_decode_attention(s["q"], s["key"], s["value"], st.k_cache, st.v_cache,
+                                                       s["slot_mapping"], s["block_tables"], s["context_lens"],
+                                                       out=out, workspace=ws)
+
+        for i in range(3):
+            step(i)
+        ops.check_device_errors()
+        ms = timed(step, steps) / steps
+        store_b, attn_b = step_bytes(wl, 0)
+        gbs = (store_b + attn_b) / (ms * 1e-3) / 1e9
+        r = {"metric": metric_for(wl), "ms_per_step": ms, "gb_s": gbs, "frac_of_hbm": gbs / hbm_peak,
+             "tokens_per_s": wl.total_q / (ms * 1e-3), "config": workload_config(wl)}
+        if wl.spec.share_group:
+            _, logical = step_bytes(wl, 0, logical=True)
+            r["logical_gb_s"] = (store_b + logical) / (ms * 1e-3) / 1e9
+            r["bytes"] = "gb_s counts each prefix-shared block once; logical_gb_s once per reading sequence"
+        if mixed:
+            r.update(mixed_subbatches(steps, wl, st, dev, stream, ops, W, timed))
+        ops.check_device_errors()
+        res[name] = r
+        del st, ws, out, s
+        torch.cuda.empty_cache()
+    return res
+
+
 def step_fn_kind(args, mixed):
     return "mixed" if mixed else ("separate" if args.separate_store else "fused")
 
 
-def mixed_subbatches(args, wl, st, dev, stream, ops, W, timed):
+def mixed_subbatches(steps, wl, st, dev, stream, ops, W, timed):
     """Time the prefill-only and decode-only parts of the mixed batch as their own calls."""
     import torch
 
@@ -602,7 +668,7 @@ def mixed_subbatches(args, wl, st, dev, stream, ops, W, timed):
 
         for i in range(3):
             call(i)
-        ms = timed(call, args.steps) / args.steps
+        ms = timed(call, steps) / steps
         _, nbytes = step_bytes(wl, 0, seqs)
         fl = prefill_flops(wl, 0, seqs)
         res[kind] = {"ms": ms, "gb_s": nbytes / (ms * 1e-3) / 1e9, "tflop_s": fl / (ms * 1e-3) / 1e12,
@@ -617,6 +683,8 @@ def mixed_subbatches(args, wl, st, dev, stream, ops, W, timed):
         roof = {"kernel": name, "bound": "tensor", "achieved": pre["tflop_s"], "peak": tflops_peak,
                 "unit": "TFLOP/s", "frac": pre["tflop_s"] / tflops_peak, "peak_source": tf_kind,
                 "traffic": traffic,
+                "traffic_source": (f"copied from the ncu capture in profiles/prefill_attention_{wl.spec.name}.txt "
+                                   "(kept only while the kernel source hash matches the capture's)"),
                 "algorithmic_flops_per_launch": prefill_flops(wl, 0, pre_seqs), "mean_launch_ms": pre["ms"]}
     else:
         roof = {"kernel": name, "bound": "hbm", "achieved": pre["gb_s"], "peak": hbm_peak, "unit": "GB/s",
@@ -630,51 +698,98 @@ def mixed_subbatches(args, wl, st, dev, stream, ops, W, timed):
 
 
 def npv_e2e(args, wl, st, ws, dev, stream, ops, W, barrier, max_over_ranks, kind):
-    """Host-resident inputs: each step copies its inputs H2D from pinned memory,
-    runs the step through the public API, and copies the output D2H."""
+    """End to end through the public API with host-resident inputs and outputs.
+
+    Each step's inputs (q, the new K/V rows and the metadata) sit packed in one
+    pinned host buffer; every step copies its buffer to the device with one
+    host-to-device copy, runs the step's library calls on views of the device
+    buffer, and copies the output back with one device-to-host copy.  The
+    copies run on their own streams, double-buffered, so step i+1's upload and
+    step i-1's download overlap step i's kernels; every copy of every timed
+    step lies inside the timed region."""
     import torch
 
     nsteps = wl.spec.num_steps
     keys = ["q", "key", "value", "slot_mapping", "block_tables", "context_lens", "cu_seqlens_q"]
+    used = keys if kind == "mixed" else keys[:-1]
+    layout, off = [], 0
+    for k in used:
+        t = st.steps[0][k]
+        nb = t.numel() * t.element_size()
+        layout.append((k, off, nb, t.dtype, tuple(t.shape)))
+        off = (off + nb + 255) // 256 * 256
+    total = off
     host = []
     for i in range(nsteps):
-        s = st.steps[i]
-        host.append({k: s[k].cpu().pin_memory() for k in keys})
-    dbuf = {k: torch.empty_like(st.steps[0][k]) for k in keys}
-    out_dev = torch.empty((wl.total_q, wl.Hq, wl.D), dtype=torch.bfloat16, device=dev)
-    out_host = torch.empty((wl.total_q, wl.Hq, wl.D), dtype=torch.bfloat16).pin_memory()
-    used = keys if kind == "mixed" else keys[:-1]
-    h2d = sum(host[0][k].numel() * host[0][k].element_size() for k in used)
-    d2h = out_host.numel() * out_host.element_size()
+        h = torch.empty(total, dtype=torch.uint8).pin_memory()
+        for k, o, nb, _, _ in layout:
+            h[o:o + nb].copy_(st.steps[i][k].contiguous().view(torch.uint8).reshape(-1).cpu())
+        host.append(h)
+    nbuf = 2
+    dbufs = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(nbuf)]
+    views = [{k: d[o:o + nb].view(dt).view(shp) for k, o, nb, dt, shp in layout} for d in dbufs]
+    out_dev = [torch.empty((wl.total_q, wl.Hq, wl.D), dtype=torch.bfloat16, device=dev) for _ in range(nbuf)]
+    out_host = [torch.empty((wl.total_q, wl.Hq, wl.D), dtype=torch.bfloat16).pin_memory() for _ in range(nbuf)]
+    h2d = total
+    d2h = out_host[0].numel() * out_host[0].element_size()
     mq = st.steps[0]["max_seqlen_q"]
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    uploaded = [ev() for _ in range(nbuf)]
+    computed = [ev() for _ in range(nbuf)]
+    downloaded = [ev() for _ in range(nbuf)]
+    started = [False] * nbuf
+
+    def compute(v, o):
+        if kind == "fused":
+            ops.store_kvcache_and_decode_attention(v["q"], v["key"], v["value"], st.k_cache, st.v_cache,
+                                                   v["slot_mapping"], v["block_tables"], v["context_lens"],
+                                                   out=o, workspace=ws)
+        else:
+            ops.store_kvcache(v["key"], v["value"], st.k_cache, st.v_cache, v["slot_mapping"])
+            if kind == "mixed":
+                ops.paged_prefill_attention(v["q"], st.k_cache, st.v_cache, v["cu_seqlens_q"], mq,
+                                            v["block_tables"], v["context_lens"], out=o, workspace=ws)
+            else:
+                ops.paged_decode_attention(v["q"], st.k_cache, st.v_cache, v["block_tables"], v["context_lens"],
+                                           out=o, workspace=ws)
 
     def step(i):
-        h = host[i % nsteps]
-        for k in used:
-            dbuf[k].copy_(h[k], non_blocking=True)
-        if kind == "fused":
-            ops.store_kvcache_and_decode_attention(dbuf["q"], dbuf["key"], dbuf["value"], st.k_cache, st.v_cache,
-                                                   dbuf["slot_mapping"], dbuf["block_tables"], dbuf["context_lens"],
-                                                   out=out_dev, workspace=ws)
-        else:
-            ops.store_kvcache(dbuf["key"], dbuf["value"], st.k_cache, st.v_cache, dbuf["slot_mapping"])
-            if kind == "mixed":
-                ops.paged_prefill_attention(dbuf["q"], st.k_cache, st.v_cache, dbuf["cu_seqlens_q"], mq,
-                                            dbuf["block_tables"], dbuf["context_lens"], out=out_dev, workspace=ws)
-            else:
-                ops.paged_decode_attention(dbuf["q"], st.k_cache, st.v_cache, dbuf["block_tables"],
-                                           dbuf["context_lens"], out=out_dev, workspace=ws)
-        out_host.copy_(out_dev, non_blocking=True)
+        j = i % nbuf
+        with torch.cuda.stream(up):
+            if started[j]:
+                up.wait_event(computed[j])  # the kernels of step i - nbuf have read this buffer
+            dbufs[j].copy_(host[i % nsteps], non_blocking=True)
+            uploaded[j].record(up)
+        stream.wait_event(uploaded[j])
+        if started[j]:
+            stream.wait_event(downloaded[j])  # step i - nbuf's output has left this buffer
+        compute(views[j], out_dev[j])
+        computed[j].record(stream)
+        with torch.cuda.stream(down):
+            down.wait_event(computed[j])
+            out_host[j].copy_(out_dev[j], non_blocking=True)
+            downloaded[j].record(down)
+        started[j] = True
+
+    def drain():
+        for j in range(nbuf):
+            if started[j]:
+                stream.wait_event(downloaded[j])
 
     for i in range(args.warmup):
         step(i)
+    drain()
     barrier()
     torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    up.wait_event(e0)
+    down.wait_event(e0)
     for i in range(args.steps):
         step(i)
+    drain()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -683,7 +798,9 @@ def npv_e2e(args, wl, st, ws, dev, stream, ops, W, barrier, max_over_ranks, kind
     world = 1 if not torch.distributed.is_initialized() else torch.distributed.get_world_size()
     return {"value": world * nbytes / (ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms / args.steps,
-            "tokens_per_s": world * args.steps * wl.total_q / (ms * 1e-3)}
+            "tokens_per_s": world * args.steps * wl.total_q / (ms * 1e-3),
+            "copies_per_step": {"h2d": 1, "d2h": 1},
+            "pipelining": "uploads and downloads on their own streams, two buffers deep"}
 
 
 def main(argv=None):

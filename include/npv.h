@@ -79,7 +79,7 @@ typedef enum {
 #define NPV_DEVERR_BLOCK_ID 0x2u    /* a live block-table entry outside [0, num_blocks) */
 #define NPV_DEVERR_CONTEXT_LEN 0x4u /* context length < 0, > max_blocks_per_seq * block_size,
                                        or smaller than the sequence's query rows */
-#define NPV_DEVERR_QUERY_LENS 0x8u  /* cu_seqlens_q not nondecreasing from 0 or past total_q */
+#define NPV_DEVERR_QUERY_LENS 0x8u  /* cu_seqlens_q not nondecreasing from 0 to total_q */
 #define NPV_DEVERR_TIMEOUT 0x10u    /* an internal pipeline wait gave up after ~2 s (library bug) */
 
 /* Static description of a status code. Never NULL. */
@@ -192,6 +192,10 @@ NPV_API size_t npv_paged_prefill_workspace_size(int32_t num_seqs, int32_t total_
  *   q             [total_q, num_q_heads, head_dim] bf16, contiguous.  Rows of
  *                 sequence b are cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1.
  *   cu_seqlens_q  [num_seqs + 1] int32 (device), nondecreasing from 0 to total_q.
+ *                 A first entry other than 0, a last entry other than total_q, or
+ *                 a decreasing entry sets NPV_DEVERR_QUERY_LENS; the rows of a
+ *                 sequence whose range is reversed or leaves [0, total_q) are
+ *                 not written.
  *                 n_b = cu_seqlens_q[b+1] - cu_seqlens_q[b] may be 0 (no rows) or
  *                 1 (a decode row).
  *   context_lens  [num_seqs] int32 (device): L_b, all cached tokens of sequence b

@@ -241,7 +241,16 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const Params p, int 
         for (int k = 0; k < nqt; ++k)
             if (pos + k < p.max_pairs) p.plan_pairs[pos + k] = make_int2(b, nqt - 1 - k);
     }
-    if (tid == 0) p.plan_count[0] = (int32_t)min(total, (long long)p.max_pairs);
+    if (tid == 0) {
+        // cu_seqlens_q must run from 0 to total_q; a list of row tiles longer than
+        // the plan can hold means ranges overlap (some entry decreased).  Either
+        // way the call's rows are not a partition of q: report it.  The plan is
+        // clamped, so no access leaves the workspace.
+        if (__ldg(p.cu_seqlens_q) != 0 || __ldg(p.cu_seqlens_q + p.num_seqs) != p.total_q ||
+            total > (long long)p.max_pairs)
+            report_error(NPV_DEVERR_QUERY_LENS);
+        p.plan_count[0] = (int32_t)min(total, (long long)p.max_pairs);
+    }
 }
 
 // ---------------------------------------------------------------------------

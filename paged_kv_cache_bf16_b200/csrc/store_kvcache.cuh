@@ -37,6 +37,10 @@ constexpr int kVecsPerThread = 4;
 // Grid-stride over (token, vector) pairs; the K and V copies of one vector are
 // issued together so each thread has 2 * kVecsPerThread loads in flight.
 __global__ void __launch_bounds__(kThreads) store_kvcache_kernel(const Params p) {
+    // Launched with programmatic stream serialisation: wait until the previous
+    // grid on the stream (which may still be reading the cache, or writing
+    // key / value / slot_mapping) has completed and its writes are visible.
+    grid_dependency_wait();
     const int64_t total = (int64_t)p.num_tokens * p.row_vecs;
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     for (int64_t base = (int64_t)blockIdx.x * kThreads * kVecsPerThread + threadIdx.x; base < total;

@@ -82,53 +82,3 @@ def oracle_compact(wl: W.Workload, step: int = 0, seqs=None, lib=None, threads: 
     cu_c[1:] = np.cumsum(wl.query_lens[seqs])
     out = O.paged_attention(qsub, kp, vp, bt_c, L[seqs], cu_c, scale=scale, threads=threads, _lib=lib)
     return out, rows
-
-
-def oracle_rows(wl: W.Workload, samples, step: int = 0, lib=None):
-    """Oracle outputs for individual packed query rows.
-
-    Row i of sequence b (n_b rows, context L_b) is computed as a one-row
-    problem over the first L_b - n_b + i + 1 tokens, which the pins show equals
-    the chunked-prefill row.  `samples` is a list of (b, i).  Returns
-    (fp64 out [len(samples), Hq, D], packed row indices).
-    """
-    from oracle import oracle as O
-
-    seqs = sorted({b for b, _ in samples})
-    L = wl.context_lens(step)
-    # pool of the sampled sequences' blocks, via the same construction as oracle_compact
-    bt = wl.block_tables(step)
-    remap = {}
-    bt_c = {}
-    for b in seqs:
-        row = np.full(wl.max_blocks_per_seq, -1, dtype=np.int32)
-        for i in range(-(-int(L[b]) // wl.BS)):
-            p = int(bt[b, i])
-            if p not in remap:
-                remap[p] = len(remap)
-            row[i] = remap[p]
-        bt_c[b] = row
-    shape = (max(1, len(remap)), wl.BS, wl.Hkv, wl.D)
-    kp = np.full(shape, W.BF16_NAN, dtype=np.uint16)
-    vp = np.full(shape, W.BF16_NAN, dtype=np.uint16)
-    for p, nv in wl.prior_fill():
-        if p in remap:
-            k, v = wl.block_contents(p, nv)
-            kp[remap[p], :nv] = k
-            vp[remap[p], :nv] = v
-    chosen = np.zeros(wl.B, dtype=bool)
-    chosen[seqs] = True
-    for s in range(step + 1):
-        seq_of_tok, _ = wl.token_positions(s)
-        keep = chosen[seq_of_tok]
-        slots = wl.slot_mapping(s)[keep]
-        k, v = wl.new_kv(s)
-        cslots = np.array([remap[int(x) // wl.BS] * wl.BS + int(x) % wl.BS for x in slots], dtype=np.int32)
-        O.store_kvcache(k[keep], v[keep], kp, vp, cslots, _lib=lib)
-    cu = wl.cu_seqlens_q()
-    q = wl.q(step)
-    rows = np.array([int(cu[b]) + i for b, i in samples], dtype=np.int64)
-    ctx = np.array([int(L[b]) - int(wl.query_lens[b]) + i + 1 for b, i in samples], dtype=np.int32)
-    btr = np.stack([bt_c[b] for b, _ in samples]).astype(np.int32)
-    out = O.decode_attention(q[rows], kp, vp, btr, ctx, _lib=lib)
-    return out, rows

@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 import torch
 
-from cases import oracle_compact, oracle_rows, tiny_spec
+from cases import oracle_compact, tiny_spec
 from gpu_common import DEV, assert_close, no_device_errors, run_store
 from paged_kv_cache_bf16_b200 import ops
 from paged_kv_cache_bf16_b200 import workloads as W
@@ -98,9 +98,10 @@ def test_prefill_chunk_split_matches_single_chunk():
     assert_close(full, ref, "single")
 
 
-def test_prefill_mixed_named_workload_sampled():
-    """The full chunked-prefill mix: 16 x 512-row chunks over priors up to 8192 plus 240
-    decode rows.  Decode rows are all checked; prefill rows are sampled."""
+def test_prefill_mixed_named_workload_all_rows():
+    """The full chunked-prefill mix: 16 x 512-row chunks over priors up to 8,192 plus 240
+    decode rows.  Every output row (8,192 prefill rows and 240 decode rows, all heads) is
+    checked element by element against the fp64 oracle."""
     wl = W.workload("chunked_prefill_mixed")
     st = W.DeviceState(wl, DEV)
     run_store(st, 0)
@@ -110,13 +111,8 @@ def test_prefill_mixed_named_workload_sampled():
     ref, rows = oracle_compact(wl, 0, seqs=dec)
     assert_close(out[torch.from_numpy(rows).to(DEV)], ref, "decode rows")
     pre = [b for b in range(wl.B) if wl.query_lens[b] > 1]
-    rng = np.random.default_rng(5)
-    samples = []
-    for b in pre:
-        n = int(wl.query_lens[b])
-        picks = {0, 1, 63, 64, 65, 127, 128, 255, 256, n - 2, n - 1} | set(rng.integers(0, n, 6).tolist())
-        samples += [(b, i) for i in sorted(picks) if i < n]
-    ref, rows = oracle_rows(wl, samples)
+    assert sum(int(wl.query_lens[b]) for b in pre) == 16 * 512
+    ref, rows = oracle_compact(wl, 0, seqs=pre)
     assert_close(out[torch.from_numpy(rows).to(DEV)], ref, "prefill rows")
 
 
@@ -163,3 +159,24 @@ def test_prefill_invalid_lengths_reported():
     assert torch.count_nonzero(out[40:80]).item() == 0
     ref, rows = oracle_compact(wl, 0, seqs=[0, 2])
     assert_close(out[torch.from_numpy(rows).to(DEV)], ref, "valid sequences")
+
+
+def test_prefill_malformed_query_ranges_reported():
+    """cu_seqlens_q that does not partition q (a reversed entry, so ranges overlap, or a
+    first entry other than 0) sets NPV_DEVERR_QUERY_LENS; the context stays usable."""
+    spec = tiny_spec(name="p_cu", seed=815, head_dim=128, num_q_heads=16, num_kv_heads=8, block_size=256,
+                     num_blocks=30, num_seqs=3, prefill_seqs=3, prefill_len=40, prior_lo=100, prior_hi=300)
+    wl = W.draw(spec)
+    st = W.DeviceState(wl, DEV)
+    run_store(st, 0)
+    s = st.steps[0]
+    for cu in ([0, 80, 40, 120], [8, 48, 88, 120]):
+        bad = torch.tensor(cu, dtype=torch.int32, device=DEV)
+        ops.paged_prefill_attention(s["q"], st.k_cache, st.v_cache, bad, 80, s["block_tables"], s["context_lens"])
+        with pytest.raises(ops.NpvError) as ei:
+            ops.check_device_errors()
+        assert ei.value.bits & 0x8, cu
+    out = run_prefill(st)
+    no_device_errors()
+    ref, rows = oracle_compact(wl, 0)
+    assert_close(out[torch.from_numpy(rows).to(DEV)], ref, "after malformed calls")
