@@ -374,9 +374,15 @@ def reference_arm(args, rank, world):
 
 def workload_config(wl):
     s = wl.spec
+    if s.prefill_seqs:
+        lens = (f"{s.prefill_seqs} sequences x {s.prefill_len} query rows over prior U[{s.prior_lo},{s.prior_hi}]"
+                + (f" + {s.num_seqs - s.prefill_seqs} decode rows over U[{s.ctx_lo},{s.ctx_hi}]"
+                   if s.num_seqs > s.prefill_seqs else ""))
+    else:
+        lens = f"U[{s.ctx_lo},{s.ctx_hi}]" + (" +1 per step" if s.num_steps > 1 else "")
     return {"workload": s.name, "num_seqs": s.num_seqs, "num_q_heads": s.num_q_heads,
             "num_kv_heads": s.num_kv_heads, "head_dim": s.head_dim, "block_size": s.block_size,
-            "num_blocks": s.num_blocks, "context_lens": f"U[{s.ctx_lo},{s.ctx_hi}] +1 per step",
+            "num_blocks": s.num_blocks, "context_lens": lens,
             "steps_cycle": s.num_steps,
             "l2": "not flushed: inputs larger than L2 (K/V read per step %.2f GB vs 126 MB L2)"
                   % (step_bytes(wl, 0)[1] / 1e9)}
@@ -687,8 +693,11 @@ def mixed_subbatches(steps, wl, st, dev, stream, ops, W, timed):
                                    "(kept only while the kernel source hash matches the capture's)"),
                 "algorithmic_flops_per_launch": prefill_flops(wl, 0, pre_seqs), "mean_launch_ms": pre["ms"]}
     else:
+        _, hbm_kind = measured_peaks()
         roof = {"kernel": name, "bound": "hbm", "achieved": pre["gb_s"], "peak": hbm_peak, "unit": "GB/s",
-                "frac": pre["gb_s"] / hbm_peak, "peak_source": "measured: MEASURED_PEAKS.json hbm_gbs",
+                "frac": pre["gb_s"] / hbm_peak,
+                "peak_source": "measured: MEASURED_PEAKS.json hbm_gbs" if hbm_kind == "measured"
+                else "fallback 6650 GB/s",
                 "traffic": None, "algorithmic_bytes_per_launch": step_bytes(wl, 0, pre_seqs)[1],
                 "mean_launch_ms": pre["ms"]}
     out = {"roofline": roof, "prefill_part": pre}

@@ -141,8 +141,10 @@ NPV_API size_t npv_paged_decode_workspace_size(int32_t num_seqs, int32_t num_q_h
  *                 once must not share a workspace.
  * Work is split over the device's SMs by KV tokens (split-KV): a sequence whose
  * tokens land on several CTAs is combined by a merge kernel from its partial
- * (max, sum, unnormalised output) triples.  Accumulation is fp32; the output is
- * rounded once to bf16 (round to nearest even).
+ * (max, sum, unnormalised output) triples.  Q K^T and P V run on warp-level
+ * tensor-core MMAs with fp32 accumulation (the probabilities P are rounded to
+ * bf16 for the P V product and the row sums add the rounded values); the
+ * output is rounded once to bf16 (round to nearest even).
  */
 NPV_API npv_status npv_paged_decode_attention(void *out, const void *q, int64_t q_seq_stride, const void *k_cache,
                                       const void *v_cache, const int32_t *block_tables,
@@ -203,12 +205,17 @@ NPV_API size_t npv_paged_prefill_workspace_size(int32_t num_seqs, int32_t total_
  *                 Row i of sequence b sits at position L_b - n_b + i and sees
  *                 keys 0 .. L_b - n_b + i.  L_b < n_b sets NPV_DEVERR_CONTEXT_LEN.
  *   max_seqlen_q  host upper bound on n_b, the flash-attn-style hint; checked to be
- *                 >= 0 and otherwise unused (the plan kernel reads the row counts
- *                 on the device).
+ *                 >= 0.  When max_seqlen_q * g <= 8 the short sequences run on a
+ *                 lighter variant of the decode kernel (see below); the row
+ *                 counts themselves are read on the device, so a wrong hint
+ *                 changes only which kernel serves a sequence, not the result.
  *   other arguments as for npv_paged_decode_attention.
- * Rows with n_b >= 2 run on the tcgen05 tensor cores (QK^T and PV with fp32
- * accumulators in tensor memory; P rounded to bf16 for the PV product); rows
- * with n_b == 1 run on the split-KV decode path within the same call.
+ * Sequences with n_b > m (g = num_q_heads / num_kv_heads; m = 8 / g when
+ * max_seqlen_q * g <= 8, else 16 / g) run on the tcgen05 tensor cores (QK^T and
+ * PV with fp32 accumulators in tensor memory); sequences with 1 <= n_b <= m
+ * (decode rows, speculative-decode verification) run on the split-KV decode
+ * kernel within the same call, whose warp-level MMA tiles hold the g * n_b rows
+ * of one KV head.  Both round P to bf16 for the PV product.
  */
 NPV_API npv_status npv_paged_prefill_attention(void *out, const void *q, const int32_t *cu_seqlens_q,
                                        int32_t max_seqlen_q, int32_t total_q, const void *k_cache,
@@ -251,6 +258,21 @@ NPV_API npv_status npv_paged_decode_attention_noalloc(void *out, const void *q, 
                                                       int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                                       int32_t num_blocks, int32_t block_size, float scale,
                                                       npv_stream_t stream);
+
+/*
+ * Test hook for failure detection; the pages have no counterpart.  With
+ * enable != 0, later decode-kernel launches on the current device (the decode
+ * calls, and the short sequences of a prefill call) run with one pipeline stage
+ * per CTA left unfilled on purpose, and their consumer warps wait for a stage at
+ * most about a millisecond instead of 2 s.  The wait therefore gives up: the
+ * kernel records NPV_DEVERR_TIMEOUT, waits (bounded, 2 s) for the copies it did
+ * issue, and returns; the outputs of such calls are meaningless, nothing
+ * faults, and the CUDA context stays usable.  npv_check_device_errors() then
+ * reports the timeout.  enable == 0 restores normal operation.  The setting is
+ * copied to the device synchronously; change it only while no call is in
+ * flight.  Returns NPV_ERR_CUDA if the copy fails.
+ */
+NPV_API npv_status npv_debug_inject_decode_timeout(int enable);
 
 /*
  * Synchronise `stream`, then read and clear the device error word of the

@@ -22,12 +22,21 @@
 //     32-entry window at a time.  HC consumer warps each own one KV head and
 //     all g query heads that share it, so every K/V row read from HBM feeds g
 //     query heads.
-//   * A consumer warp reads 16-byte rows from shared memory (D/8 lanes per row,
-//     conflict-free), forms partial dot products, reduce-scatters them across
-//     the row's lanes so that each lane ends with one token's score per head,
-//     and runs an fp32 online softmax in the log2 domain (scale * log2 e is
-//     folded into q).  Probabilities pass through a per-warp shared buffer to
-//     the P.V step, which accumulates an 8-element slice of the output per lane.
+//   * A consumer warp runs both products of a chunk on the warp-level tensor
+//     cores (mma.sync m16n8k16, bf16 in, fp32 accumulate), with the chunk's 16
+//     tokens as the MMA's M and the query rows sharing the warp's KV head as
+//     its N: the g heads of a GQA group times the sequence's n query rows
+//     (n = 1 for decode; up to 16 / g for speculative-decode verification or a
+//     short chunk), in one or two 8-column tiles, unused columns zero.
+//     S^T = K Q^T takes D / 16 MMAs per tile; after the online softmax (log2
+//     domain, running max and sum per row) and a bf16 rounding, movmatrix
+//     transposes the accumulator into the B operand of O^T += V^T P^T (D / 16
+//     MMAs per tile), so P never leaves registers.  Lanes read K and V rows
+//     from shared memory with 16-byte loads: the head dimension inside a K
+//     fragment follows a fixed permutation shared by Q (the dot product does
+//     not depend on it) so the loads are contiguous, and V is transposed into
+//     A fragments with byte permutes.  A row's causal limit is L - n + i for
+//     its query row i.
 #pragma once
 
 #include "npv_device.cuh"
@@ -40,14 +49,24 @@ constexpr int kMaxConsumerWarps = 8;
 constexpr int kMaxStages = 8;
 constexpr int kStageBudgetBytes = 192 * 1024;
 constexpr int kHeaderBytes = 1024;
+constexpr int kTileRows = 16;              // most query rows per KV head: two 8-column MMA tiles
+constexpr float kRescaleThreshold = 8.0f;  // log2 units a row max may grow before O is rescaled
 
 enum : int32_t { kFlagFirst = 1, kFlagLast = 2, kFlagSkip = 4, kFlagNewToken = 8 };
+
+// Failure-detection test hook (npv_debug_inject_decode_timeout), off unless the
+// host sets it: every CTA's producer leaves its first stage unfilled, and the
+// consumers wait for a stage at most kDebugWaitNs, so their wait certainly gives
+// up, records NPV_DEVERR_TIMEOUT and ends the kernel through its exit path.
+__device__ unsigned int g_debug_timeout;
+constexpr uint64_t kDebugWaitNs = 1000000ull;
 
 struct StageInfo {
     int32_t unit;     // (sequence, head group) index
     int32_t n_valid;  // live tokens in the chunk (1..16)
     int32_t flags;
     int32_t slot;  // partial slot written at kFlagLast, or -1 for a finished unit
+    int32_t tok0;  // position of the chunk's first token in its sequence
 };
 
 struct Params {
@@ -58,8 +77,10 @@ struct Params {
     const uint16_t *v_cache;
     const int32_t *block_tables;
     const int32_t *context_lens;
-    const int32_t *cu_seqlens_q;  // non-null: mixed batch; only sequences with one query row run here
+    const int32_t *cu_seqlens_q;  // non-null: mixed batch; sequences with 1..max_rows query rows run here
     int32_t total_q;              // rows of q and out in a mixed batch
+    int32_t max_rows;             // most query rows of a sequence on this path (1 without cu_seqlens_q)
+    int32_t rows_per_head;        // RP: query-row slots per KV head in a partial slot (g * max_rows)
     int32_t max_blocks_per_seq;
     int32_t num_seqs;
     int32_t num_q_heads;
@@ -78,19 +99,28 @@ struct Params {
     int64_t value_stride;
     const int32_t *slot_mapping;
     // workspace
-    float2 *part_ml;  // [grid][2][HC*g]: (running max, sum) of a partial unit
-    float *part_o;    // [grid][2][HC*g][D]: unnormalised output of a partial unit
+    float2 *part_ml;  // [grid][2][HC][RP]: (running max, sum) of a partial unit's rows
+    float *part_o;    // [grid][2][HC][RP][D]: unnormalised output of a partial unit's rows
 };
 
+// Query rows of sequence b on this path: 1 in a decode call; in a mixed batch
+// n_b when 1 <= n_b <= max_rows, else 0 (no rows, a malformed range, or a
+// sequence the prefill kernel serves).
+__device__ __forceinline__ int32_t path_rows(const Params &p, int32_t b) {
+    if (p.cu_seqlens_q == nullptr) return 1;
+    const int32_t cb = __ldg(p.cu_seqlens_q + b), ce = __ldg(p.cu_seqlens_q + b + 1);
+    const int32_t n = ce - cb;
+    if (cb < 0 || ce > p.total_q || n < 1 || n > p.max_rows) return 0;
+    return n;
+}
+
 // Chunks of work for sequence b on this path (0 for an empty, invalid or
-// multi-row sequence; the merge kernel writes those rows or reports them).
+// foreign sequence; the merge kernel writes those rows or reports them).
 __device__ __forceinline__ int32_t seq_chunks(const Params &p, int32_t b) {
+    const int32_t n = path_rows(p, b);
+    if (n == 0) return 0;
     const int32_t L = __ldg(p.context_lens + b);
-    if (p.cu_seqlens_q != nullptr) {
-        const int32_t cb = __ldg(p.cu_seqlens_q + b), ce = __ldg(p.cu_seqlens_q + b + 1);
-        if (ce - cb != 1 || cb < 0 || ce > p.total_q) return 0;
-    }
-    if (L <= 0 || (long long)L > (long long)p.max_blocks_per_seq * p.block_size) return 0;
+    if (L < n || (long long)L > (long long)p.max_blocks_per_seq * p.block_size) return 0;
     return (L + kChunk - 1) / kChunk;
 }
 
@@ -188,36 +218,52 @@ __device__ __forceinline__ void store_token_rows(const Params &p, int32_t b, int
     }
 }
 
-template <int D, int G>
-struct Shape {
-    static constexpr int LPR = D / 8;          // lanes per 16-byte-vector row
-    static constexpr int RPL = 32 / LPR;       // rows per warp-wide load
-    static constexpr int NI = kChunk / RPL;    // warp-wide loads per stage
-    static constexpr int LOG_NI = NI == 8 ? 3 : (NI == 4 ? 2 : 1);
-};
+// D[16 x 8] += A[16 x 16] B[16 x 8]: bf16 inputs, fp32 accumulators, one warp.
+// Fragments follow the PTX ISA's m16n8k16 layout: lane = 4 * group + t holds
+// A rows group and group + 8, columns 2t, 2t + 1 (a0, a1) and 2t + 8, 2t + 9
+// (a2, a3); B column group, rows 2t, 2t + 1 (b0) and 2t + 8, 2t + 9 (b1);
+// D rows group (d0, d1) and group + 8 (d2, d3), columns 2t, 2t + 1.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 
-// Consumer warps (= KV heads) per CTA: 8, or 4 when g = 8 so that the larger
-// per-thread state (8 query heads) fits in registers.
-__host__ __device__ constexpr int max_heads_per_cta(int g) { return g >= 8 ? 4 : kMaxConsumerWarps; }
+__device__ __forceinline__ void swap_if(uint4 &a, uint4 &b, bool c) {
+    const uint4 x = a, y = b;
+    a = c ? y : x;
+    b = c ? x : y;
+}
 
-template <int D, int G>
-__global__ void __launch_bounds__((max_heads_per_cta(G) + 1) * 32, 1) decode_split_kernel(const Params p) {
-    using S = Shape<D, G>;
+__device__ __forceinline__ uint32_t word(const uint4 &v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
+
+// Transpose of an 8 x 8 matrix of 16-bit elements held one 32-bit pair per lane
+// (lane 4 r + c holds row r, columns 2c, 2c + 1).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+    uint32_t y;
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+// NR: tiles of 8 query rows per KV head (1: g * n <= 8, as in every decode call;
+// 2: up to 16 rows, for the short sequences of a prefill call).
+template <int D, int G, int NR>
+__global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1) decode_split_kernel(const Params p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem);
     uint64_t *empty_bar = full_bar + kMaxStages;
     StageInfo *info = reinterpret_cast<StageInfo *>(empty_bar + kMaxStages);
     long long *sched = reinterpret_cast<long long *>(info + kMaxStages);  // [0..7]
     long long *scan_scratch = sched + 8;                                  // [kMaxConsumerWarps + 2]
-    float *pbuf = reinterpret_cast<float *>(smem + kHeaderBytes);         // [HC][kChunk][G]
 
     const int HC = p.heads_per_cta;
     const int NS = p.num_stages;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int pbuf_bytes = ((HC * kChunk * G * 4) + 1023) & ~1023;
     const int row_elems = HC * D;  // one token of one head group
     const int stage_elems = kChunk * row_elems;
-    uint16_t *stage_k = reinterpret_cast<uint16_t *>(smem + kHeaderBytes + pbuf_bytes);
+    uint16_t *stage_k = reinterpret_cast<uint16_t *>(smem + kHeaderBytes);
     uint16_t *stage_v = stage_k + (size_t)NS * stage_elems;
 
     if (threadIdx.x == 0) {
@@ -240,8 +286,10 @@ __global__ void __launch_bounds__((max_heads_per_cta(G) + 1) * 32, 1) decode_spl
     const long long u_first = sc.u_first;
     const long long s_first = sc.s_first;
 
+    const bool debug_timeout = *reinterpret_cast<volatile unsigned int *>(&g_debug_timeout) != 0;
     if (warp == HC) {
         // ===================== producer warp =====================
+        bool drop = debug_timeout;  // leave the first stage unfilled (test hook)
         long long remaining = c1 - c0;
         long long u = u_first;
         long long k = c0 - s_first;
@@ -283,6 +331,15 @@ __global__ void __launch_bounds__((max_heads_per_cta(G) + 1) * 32, 1) decode_spl
                     abort = true;
                     break;
                 }
+                if (drop) {
+                    // test hook: no copy and no arrival, so this stage never fills
+                    drop = false;
+                    if (++stage == NS) {
+                        stage = 0;
+                        eparity ^= 1;
+                    }
+                    continue;
+                }
                 if (lane == 0) {
                     int32_t flags = (i == 0 ? kFlagFirst : 0) | (i == seg_len - 1 ? kFlagLast : 0);
                     // a fused store: this segment ends with the unit's last chunk, which
@@ -292,7 +349,7 @@ __global__ void __launch_bounds__((max_heads_per_cta(G) + 1) * 32, 1) decode_spl
                         flags |= kFlagSkip;
                         report_error(NPV_DEVERR_BLOCK_ID);
                     }
-                    info[stage] = StageInfo{(int32_t)u, n_valid, flags, slot};
+                    info[stage] = StageInfo{(int32_t)u, n_valid, flags, slot, t0};
                     if (valid)
                         mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)(2 * n_valid * row_elems * 2));
                     else
@@ -340,43 +397,80 @@ __global__ void __launch_bounds__((max_heads_per_cta(G) + 1) * 32, 1) decode_spl
     }
 
     // ===================== consumer warps (one KV head each) =====================
-    constexpr int LPR = S::LPR, RPL = S::RPL, NI = S::NI;
-    const int rg = lane / LPR;   // which row of a warp-wide load this lane reads
-    const int sub = lane % LPR;  // which 8-element slice of the row
-    const int HCG = HC * G;
-    float *my_p = pbuf + warp * (kChunk * G);
-    const uint32_t k_lane = smem_addr(stage_k) + (uint32_t)((warp * D + sub * 8) * 2);
-    const uint32_t v_lane = smem_addr(stage_v) + (uint32_t)((warp * D + sub * 8) * 2);
+    // Per 16-token chunk, with the chunk's tokens as MMA rows and the query rows
+    // as MMA columns (NR tiles of 8):
+    //   S^T = K Q^T       (D / 16 k-steps per 8 query rows)
+    //   O^T += V^T P^T    (D / 16 tiles of 16 output dims per 8 query rows)
+    // The S^T accumulator of lane (group, t) holds query rows 2t, 2t + 1 at
+    // tokens group and group + 8; after the softmax, each bf16 pair of it is one
+    // lane's share of an 8 x 8 block of P^T, and movmatrix's transpose turns the
+    // two blocks into the B fragment of P^T.
+    constexpr int KJ = D / 32;   // 16-byte K vectors a lane reads per token row
+    constexpr int VH = D / 64;   // 16-byte V vectors a lane reads per token row
+    constexpr int MT = D / 16;   // 16-dim tiles of the output
+    const int gq = lane >> 2, tq = lane & 3;
     const uint32_t tok_bytes = (uint32_t)(row_elems * 2);
     const uint32_t stage_bytes = (uint32_t)(stage_elems * 2);
+    // K fragment: tokens gq and gq + 8, vector j holding dims 32 j + 8 tq .. + 7 (a
+    // fixed permutation of the head dim inside each k-step pair, shared by Q).
+    // Lanes with odd gq read the two vectors of a pair in the other order, so a
+    // quarter-warp's loads hit distinct banks, and swap them back in registers.
+    const uint32_t k_lane = smem_addr(stage_k) + (uint32_t)(warp * D * 2) + (uint32_t)gq * tok_bytes + 16u * tq;
+    const bool k_odd = KJ > 1 && (gq & 1);
+    // V fragment: tokens 2 tq, 2 tq + 1, 2 tq + 8, 2 tq + 9 at dims (D / 8) gq .. + D / 8 - 1;
+    // output tile mt's rows gq and gq + 8 are dims (D / 8) gq + mt and + D / 16 + mt.
+    const uint32_t v_lane = smem_addr(stage_v) + (uint32_t)(warp * D * 2) + (uint32_t)(2 * tq) * tok_bytes +
+                            (uint32_t)(2 * (D / 8) * gq);
+    const bool v_odd = VH > 1 && (tq & 1);
 
-    float qf[G][8], o[G][8], m_run[G], l_run[G];
-    int32_t b = 0, hg = 0;
+    uint4 qf[NR][KJ];  // query row 8 nr + gq, vectors as K's
+    float o[NR][MT][4];
+    float m_run[NR][2], l_run[NR][2];
+    int32_t lim[NR][2];
+    int32_t b = 0, hg = 0, R = 0, lim_min = 0;
+    int64_t row0 = 0;
     // fused store: this lane's 8-element slices of the new token's K and V rows
     uint4 new_k = make_uint4(0, 0, 0, 0), new_v = make_uint4(0, 0, 0, 0);
     int32_t new_slot = -1;
     int stage = 0;
     uint32_t fparity = 0;
+    const float sl2 = p.scale_log2;
     const long long nchunks = c1 - c0;
+    const uint64_t wait_ns = debug_timeout ? kDebugWaitNs : kWaitLimitNs;
     for (long long it = 0; it < nchunks; ++it) {
-        if (!mbar_wait(&full_bar[stage], fparity)) break;
+        if (!mbar_wait(&full_bar[stage], fparity, wait_ns)) break;
         const StageInfo inf = info[stage];
         if (inf.flags & kFlagFirst) {
             b = inf.unit / NHG;
             hg = inf.unit % NHG;
-            const uint16_t *qrow = p.q + query_row(p, b) * p.q_row_stride +
-                                   ((int64_t)(hg * HC + warp) * G) * D + sub * 8;
+            const int32_t n = path_rows(p, b);
+            const int32_t L = __ldg(p.context_lens + b);
+            R = G * n;
+            row0 = query_row(p, b);
+            lim_min = L - n;
 #pragma unroll
-            for (int j = 0; j < G; ++j) {
-                float f[8];
-                unpack8(ld_nc_v4(qrow + j * D), f);
+            for (int nr = 0; nr < NR; ++nr) {
+                const int r = 8 * nr + gq;
+                if (r < R) {
+                    const uint16_t *qrow = p.q + (row0 + r / G) * p.q_row_stride +
+                                           ((int64_t)(hg * HC + warp) * G + r % G) * D + 8 * tq;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    qf[j][e] = f[e] * p.scale_log2;
-                    o[j][e] = 0.f;
+                    for (int j = 0; j < KJ; ++j) qf[nr][j] = ld_nc_v4(qrow + 32 * j);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < KJ; ++j) qf[nr][j] = make_uint4(0, 0, 0, 0);
                 }
-                m_run[j] = -INFINITY;
-                l_run[j] = 0.f;
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    // row i of the sequence sees keys 0 .. L - n + i; rows past R (never
+                    // stored) attend like the unit's last row
+                    const int rr = 8 * nr + 2 * tq + u;
+                    lim[nr][u] = rr < R ? L - n + rr / G : L - 1;
+                    m_run[nr][u] = -INFINITY;
+                    l_run[nr][u] = 0.f;
+                }
+#pragma unroll
+                for (int i = 0; i < MT; ++i) o[nr][i][0] = o[nr][i][1] = o[nr][i][2] = o[nr][i][3] = 0.f;
             }
             new_slot = -1;
             if (inf.flags & kFlagNewToken) {
@@ -384,9 +478,11 @@ __global__ void __launch_bounds__((max_heads_per_cta(G) + 1) * 32, 1) decode_spl
                 const int32_t slot = __ldg(p.slot_mapping + b);
                 if (slot >= 0 && (long long)slot < (long long)p.num_blocks * p.block_size) {
                     new_slot = slot;
-                    const int64_t h = (int64_t)(hg * HC + warp) * D + sub * 8;
-                    new_k = ld_nc_v4(p.key + (int64_t)b * p.key_stride + h);
-                    new_v = ld_nc_v4(p.value + (int64_t)b * p.value_stride + h);
+                    if (lane < D / 8) {
+                        const int64_t h = (int64_t)(hg * HC + warp) * D + lane * 8;
+                        new_k = ld_nc_v4(p.key + (int64_t)b * p.key_stride + h);
+                        new_v = ld_nc_v4(p.value + (int64_t)b * p.value_stride + h);
+                    }
                 } else if (slot >= 0 && lane == 0) {
                     report_error(NPV_DEVERR_SLOT);
                 }
@@ -395,9 +491,8 @@ __global__ void __launch_bounds__((max_heads_per_cta(G) + 1) * 32, 1) decode_spl
         if ((inf.flags & kFlagLast) && new_slot >= 0) {
             // the unit's last chunk: put the new token into the stage (its cache
             // slot may not hold it yet) and into the cache
-            const int tl = inf.n_valid - 1;
-            if (rg == 0) {
-                const uint32_t off = (uint32_t)(((tl * HC + warp) * D + sub * 8) * 2);
+            if (lane < D / 8) {
+                const uint32_t off = (uint32_t)((((inf.n_valid - 1) * HC + warp) * D + lane * 8) * 2);
                 asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_addr(stage_k) + stage * stage_bytes +
                                                                             off),
                              "r"(new_k.x), "r"(new_k.y), "r"(new_k.z), "r"(new_k.w)
@@ -406,108 +501,133 @@ __global__ void __launch_bounds__((max_heads_per_cta(G) + 1) * 32, 1) decode_spl
                                                                             off),
                              "r"(new_v.x), "r"(new_v.y), "r"(new_v.z), "r"(new_v.w)
                              : "memory");
-                const int64_t dst = ((int64_t)new_slot * p.num_kv_heads + hg * HC + warp) * D + sub * 8;
+                const int64_t dst = ((int64_t)new_slot * p.num_kv_heads + hg * HC + warp) * D + lane * 8;
                 st_global_v4(const_cast<uint16_t *>(p.k_cache) + dst, new_k);
                 st_global_v4(const_cast<uint16_t *>(p.v_cache) + dst, new_v);
             }
             __syncwarp();
         }
         if (!(inf.flags & kFlagSkip)) {
-            const bool full = inf.n_valid == kChunk;
-            const uint32_t kst = k_lane + stage * stage_bytes;
-            const uint32_t vst = v_lane + stage * stage_bytes;
-            // ---- scores: partial dot products of this lane's 8 dims
-            float acc[NI][G];
+            const int nr_live = R > 8 ? NR : 1;  // warp-uniform
+            // ---- S^T = K Q^T
+            const uint32_t ks = k_lane + stage * stage_bytes;
+            uint4 kv[2][KJ];
 #pragma unroll
-            for (int i = 0; i < NI; ++i) {
-                float kf[8];
-                unpack8(ld_shared_v4(kst + (uint32_t)(i * RPL + rg) * tok_bytes), kf);
+            for (int mh = 0; mh < 2; ++mh)
 #pragma unroll
-                for (int j = 0; j < G; ++j) {
-                    // even and odd dims accumulate in the two halves of a pair
-                    float2 a = fmul2(make_float2(qf[j][0], qf[j][1]), make_float2(kf[0], kf[1]));
+                for (int j = 0; j < KJ; ++j)
+                    kv[mh][j] = ld_shared_v4(ks + (uint32_t)(mh * 8) * tok_bytes + (uint32_t)((64 * j) ^ (k_odd ? 64 : 0)));
+            if (KJ > 1) {
 #pragma unroll
-                    for (int e = 2; e < 8; e += 2)
-                        a = ffma2(make_float2(qf[j][e], qf[j][e + 1]), make_float2(kf[e], kf[e + 1]), a);
-                    acc[i][j] = a.x + a.y;
-                }
+                for (int mh = 0; mh < 2; ++mh)
+#pragma unroll
+                    for (int j = 0; j < KJ; j += 2) swap_if(kv[mh][j], kv[mh][j + 1], k_odd);
             }
-            // ---- reduce-scatter over the row's lanes: halve the token list at
-            // each step, keeping the half selected by this lane's bit
+            float x[NR][4];
 #pragma unroll
-            for (int step = 0; step < S::LOG_NI; ++step) {
-                const int n = NI >> (step + 1);
-                const int mask = LPR >> (step + 1);
-                const bool upper = (sub & mask) != 0;
+            for (int nr = 0; nr < NR; ++nr) {
+                x[nr][0] = x[nr][1] = x[nr][2] = x[nr][3] = 0.f;
+                if (nr < nr_live) {
+                    // vector j, elements 0-3: k-step 2 j; elements 4-7: k-step 2 j + 1
 #pragma unroll
-                for (int i = 0; i < n; ++i) {
-#pragma unroll
-                    for (int j = 0; j < G; ++j) {
-                        const float send = upper ? acc[i][j] : acc[i + n][j];
-                        const float keep = upper ? acc[i + n][j] : acc[i][j];
-                        acc[i][j] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+                    for (int j = 0; j < KJ; ++j) {
+                        mma_16816(x[nr], kv[0][j].x, kv[1][j].x, kv[0][j].y, kv[1][j].y, qf[nr][j].x, qf[nr][j].y);
+                        mma_16816(x[nr], kv[0][j].z, kv[1][j].z, kv[0][j].w, kv[1][j].w, qf[nr][j].z, qf[nr][j].w);
                     }
                 }
             }
-            float s[G];
+            // ---- online softmax (log2 domain) per query row; x[nr][c]: row 8 nr + 2 tq + (c & 1),
+            // token gq + 8 (c >> 1)
+            const bool masked = inf.n_valid < kChunk || inf.tok0 + kChunk - 1 > lim_min;
+            uint32_t pb[NR][2];
 #pragma unroll
-            for (int j = 0; j < G; ++j) {
-                float v = acc[0][j];
+            for (int nr = 0; nr < NR; ++nr) {
+                pb[nr][0] = pb[nr][1] = 0u;
+                if (nr >= nr_live) continue;
 #pragma unroll
-                for (int mask = (LPR >> (S::LOG_NI + 1)); mask >= 1; mask >>= 1)
-                    v += __shfl_xor_sync(0xffffffffu, v, mask);
-                s[j] = v;
-            }
-            // this lane now holds the score of token (sub >> 1) * RPL + rg
-            const int my_tok = (sub >> 1) * RPL + rg;
-            if (!full && my_tok >= inf.n_valid) {
+                for (int c = 0; c < 4; ++c) x[nr][c] *= sl2;
+                if (masked) {
 #pragma unroll
-                for (int j = 0; j < G; ++j) s[j] = -INFINITY;
-            }
-            // ---- online softmax (log2 domain); the running max is warp-uniform
-            float pj[G];
-#pragma unroll
-            for (int j = 0; j < G; ++j) {
-                float mx = s[j];
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                if (mx > m_run[j]) {
-                    const float alpha = fast_exp2(m_run[j] - mx);
-                    l_run[j] *= alpha;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) o[j][e] *= alpha;
-                    m_run[j] = mx;
-                }
-                pj[j] = fast_exp2(s[j] - m_run[j]);
-                l_run[j] += pj[j];
-            }
-            __syncwarp();
-            if ((lane & 1) == 0) {
-#pragma unroll
-                for (int j = 0; j < G; ++j) my_p[my_tok * G + j] = pj[j];
-            }
-            __syncwarp();
-            // ---- o += p . V over this lane's tokens and 8 dims
-#pragma unroll
-            for (int i = 0; i < NI; ++i) {
-                const int tok = i * RPL + rg;
-                if (full || tok < inf.n_valid) {
-                    float vf[8];
-                    unpack8(ld_shared_v4(vst + (uint32_t)tok * tok_bytes), vf);
-#pragma unroll
-                    for (int j = 0; j < G; ++j) {
-                        const float pv = my_p[tok * G + j];
-#pragma unroll
-                        for (int e = 0; e < 8; e += 2) {
-                            const float2 r = ffma2(make_float2(pv, pv), make_float2(vf[e], vf[e + 1]),
-                                                   make_float2(o[j][e], o[j][e + 1]));
-                            o[j][e] = r.x;
-                            o[j][e + 1] = r.y;
-                        }
+                    for (int c = 0; c < 4; ++c) {
+                        const int tok = gq + 8 * (c >> 1);
+                        if (tok >= inf.n_valid || inf.tok0 + tok > lim[nr][c & 1]) x[nr][c] = -INFINITY;
                     }
                 }
+                float mx[2] = {fmaxf(x[nr][0], x[nr][2]), fmaxf(x[nr][1], x[nr][3])};
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    mx[u] = fmaxf(mx[u], __shfl_xor_sync(0xffffffffu, mx[u], 4));
+                    mx[u] = fmaxf(mx[u], __shfl_xor_sync(0xffffffffu, mx[u], 8));
+                    mx[u] = fmaxf(mx[u], __shfl_xor_sync(0xffffffffu, mx[u], 16));
+                }
+                // lazy rescale: a row's reference max moves only when the row max
+                // grows by more than kRescaleThreshold; the final division by the
+                // row sum makes the result independent of the reference
+                const float n0 = fmaxf(m_run[nr][0], mx[0]), n1 = fmaxf(m_run[nr][1], mx[1]);
+                const bool need0 = n0 > m_run[nr][0] + kRescaleThreshold;
+                const bool need1 = n1 > m_run[nr][1] + kRescaleThreshold;
+                if (__any_sync(0xffffffffu, need0 || need1)) {
+                    const float a0 = need0 ? fast_exp2(m_run[nr][0] - n0) : 1.f;
+                    const float a1 = need1 ? fast_exp2(m_run[nr][1] - n1) : 1.f;
+                    if (need0) m_run[nr][0] = n0;
+                    if (need1) m_run[nr][1] = n1;
+                    l_run[nr][0] *= a0;
+                    l_run[nr][1] *= a1;
+#pragma unroll
+                    for (int i = 0; i < MT; ++i) {
+                        o[nr][i][0] *= a0;
+                        o[nr][i][2] *= a0;
+                        o[nr][i][1] *= a1;
+                        o[nr][i][3] *= a1;
+                    }
+                }
+                // a row with every key so far masked keeps m = -inf: its probabilities are 0
+                const float u0 = m_run[nr][0] == -INFINITY ? 0.f : m_run[nr][0];
+                const float u1 = m_run[nr][1] == -INFINITY ? 0.f : m_run[nr][1];
+                // (token gq, rows 2tq, 2tq+1) and (token gq + 8, ...): one lane's share of
+                // the two 8 x 8 blocks of P^T; transposed, the B fragment of P^T
+                const uint32_t w0 = pack_bf16x2(fast_exp2(x[nr][0] - u0), fast_exp2(x[nr][1] - u1));
+                const uint32_t w1 = pack_bf16x2(fast_exp2(x[nr][2] - u0), fast_exp2(x[nr][3] - u1));
+                // the row sums add the bf16-rounded probabilities the P V product uses
+                l_run[nr][0] += bf16lo_to_f32(w0) + bf16lo_to_f32(w1);
+                l_run[nr][1] += bf16hi_to_f32(w0) + bf16hi_to_f32(w1);
+                pb[nr][0] = movmatrix_trans(w0);
+                pb[nr][1] = movmatrix_trans(w1);
+            }
+            // ---- O^T += V^T P^T
+            const uint32_t vs = v_lane + stage * stage_bytes;
+            uint4 vv[4][VH];
+#pragma unroll
+            for (int d4 = 0; d4 < 4; ++d4)
+#pragma unroll
+                for (int h = 0; h < VH; ++h)
+                    vv[d4][h] = ld_shared_v4(vs + (uint32_t)((d4 & 1) + 8 * (d4 >> 1)) * tok_bytes +
+                                             (uint32_t)((16 * h) ^ (v_odd ? 16 : 0)));
+            if (VH > 1) {
+#pragma unroll
+                for (int d4 = 0; d4 < 4; ++d4) swap_if(vv[d4][0], vv[d4][VH - 1], v_odd);
+            }
+            if (inf.n_valid < kChunk) {
+                // rows past the chunk's tokens hold stale bytes: zero them (P is 0 there)
+#pragma unroll
+                for (int d4 = 0; d4 < 4; ++d4)
+                    if (2 * tq + (d4 & 1) + 8 * (d4 >> 1) >= inf.n_valid)
+#pragma unroll
+                        for (int h = 0; h < VH; ++h) vv[d4][h] = make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                // A = V^T tile mt: rows (dims) e0 = mt and e1 = D / 16 + mt of this lane's
+                // slice, columns (tokens) 2 tq, 2 tq + 1 and 2 tq + 8, 2 tq + 9
+                const int e0 = mt, e1 = D / 16 + mt;
+                const uint32_t s0 = (e0 & 1) ? 0x7632u : 0x5410u, s1 = (e1 & 1) ? 0x7632u : 0x5410u;
+                const uint32_t a0 = __byte_perm(word(vv[0][e0 >> 3], (e0 & 7) >> 1), word(vv[1][e0 >> 3], (e0 & 7) >> 1), s0);
+                const uint32_t a1 = __byte_perm(word(vv[0][e1 >> 3], (e1 & 7) >> 1), word(vv[1][e1 >> 3], (e1 & 7) >> 1), s1);
+                const uint32_t a2 = __byte_perm(word(vv[2][e0 >> 3], (e0 & 7) >> 1), word(vv[3][e0 >> 3], (e0 & 7) >> 1), s0);
+                const uint32_t a3 = __byte_perm(word(vv[2][e1 >> 3], (e1 & 7) >> 1), word(vv[3][e1 >> 3], (e1 & 7) >> 1), s1);
+#pragma unroll
+                for (int nr = 0; nr < NR; ++nr)
+                    if (nr < nr_live) mma_16816(o[nr][mt], a0, a1, a2, a3, pb[nr][0], pb[nr][1]);
             }
         }
         __syncwarp();
@@ -517,50 +637,41 @@ __global__ void __launch_bounds__((max_heads_per_cta(G) + 1) * 32, 1) decode_spl
             fparity ^= 1;
         }
         if (inf.flags & kFlagLast) {
-            // ---- combine the row groups, total the sums, write out or a partial
+            // ---- total the row sums over the row's 8 lanes (one per token pair); write
+            // out or a partial.  This lane holds dims (D / 8) gq + e of query rows
+            // 8 nr + 2 tq + u: o[nr][e][u] for e < D / 16, o[nr][e - D / 16][2 + u] above.
 #pragma unroll
-            for (int mask = LPR; mask < 32; mask <<= 1) {
+            for (int nr = 0; nr < NR; ++nr) {
 #pragma unroll
-                for (int j = 0; j < G; ++j)
+                for (int u = 0; u < 2; ++u) {
+                    float lt = l_run[nr][u];
+                    lt += __shfl_xor_sync(0xffffffffu, lt, 4);
+                    lt += __shfl_xor_sync(0xffffffffu, lt, 8);
+                    lt += __shfl_xor_sync(0xffffffffu, lt, 16);
+                    const int r = 8 * nr + 2 * tq + u;
+                    if (r >= R) continue;
+                    float f[D / 8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) o[j][e] += __shfl_xor_sync(0xffffffffu, o[j][e], mask);
-            }
-            float lt[G];
+                    for (int e = 0; e < D / 8; ++e) f[e] = e < D / 16 ? o[nr][e][u] : o[nr][e - D / 16][2 + u];
+                    if (inf.slot < 0) {
+                        uint16_t *orow = p.out +
+                                         ((row0 + r / G) * p.num_q_heads + (int64_t)(hg * HC + warp) * G + r % G) * D +
+                                         (D / 8) * gq;
+                        const float inv = 1.0f / lt;
 #pragma unroll
-            for (int j = 0; j < G; ++j) {
-                float v = l_run[j];
-                v += __shfl_xor_sync(0xffffffffu, v, 16);
-                v += __shfl_xor_sync(0xffffffffu, v, 8);
-                v += __shfl_xor_sync(0xffffffffu, v, 4);
-                v += __shfl_xor_sync(0xffffffffu, v, 2);
-                lt[j] = v;
-            }
-            if (inf.slot < 0) {
-                if (rg == 0) {
-                    uint16_t *orow = p.out + query_row(p, b) * (int64_t)p.num_q_heads * D +
-                                     ((int64_t)(hg * HC + warp) * G) * D + sub * 8;
+                        for (int v = 0; v < D / 64; ++v) {
+                            float w[8];
 #pragma unroll
-                    for (int j = 0; j < G; ++j) {
-                        const float inv = 1.0f / lt[j];
-                        float r[8];
+                            for (int e = 0; e < 8; ++e) w[e] = f[8 * v + e] * inv;
+                            st_global_v4(orow + 8 * v, pack8(w));
+                        }
+                    } else {
+                        const size_t pr = ((size_t)inf.slot * HC + warp) * p.rows_per_head + r;
+                        float4 *po = reinterpret_cast<float4 *>(p.part_o + pr * D + (D / 8) * gq);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) r[e] = o[j][e] * inv;
-                        st_global_v4(orow + j * D, pack8(r));
+                        for (int v = 0; v < D / 32; ++v) po[v] = make_float4(f[4 * v], f[4 * v + 1], f[4 * v + 2], f[4 * v + 3]);
+                        if (gq == 0) p.part_ml[pr] = make_float2(m_run[nr][u], lt);
                     }
-                }
-            } else {
-                if (rg == 0) {
-                    float *po = p.part_o + ((size_t)inf.slot * HCG + warp * G) * D + sub * 8;
-#pragma unroll
-                    for (int j = 0; j < G; ++j) {
-                        reinterpret_cast<float4 *>(po + j * D)[0] = make_float4(o[j][0], o[j][1], o[j][2], o[j][3]);
-                        reinterpret_cast<float4 *>(po + j * D)[1] = make_float4(o[j][4], o[j][5], o[j][6], o[j][7]);
-                    }
-                }
-                if (lane == 0) {
-#pragma unroll
-                    for (int j = 0; j < G; ++j)
-                        p.part_ml[(size_t)inf.slot * HCG + warp * G + j] = make_float2(m_run[j], lt[j]);
                 }
             }
         }
@@ -582,26 +693,24 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const Params p, int h
     const long long G = gridDim.x;
     const int HC = p.heads_per_cta;
     const int g = p.num_q_heads / p.num_kv_heads;
-    const int HCG = HC * g;
+    const int RP = p.rows_per_head;
     const int NHG = p.num_head_groups;
 
     const Schedule sc = compute_schedule(p, sched, scratch);
 
-    // (1) rows with no chunks on this path
+    // (1) rows of this path's sequences with no chunks
     for (long long b = c + G * threadIdx.x; b < p.num_seqs; b += G * blockDim.x) {
+        const int32_t n = path_rows(p, (int32_t)b);
+        // other sequences belong to the prefill kernel, which also reports
+        // malformed cu_seqlens_q
+        if (n == 0) continue;
         const int32_t L = __ldg(p.context_lens + b);
-        if (p.cu_seqlens_q != nullptr) {
-            const int32_t cb = __ldg(p.cu_seqlens_q + b), ce = __ldg(p.cu_seqlens_q + b + 1);
-            // multi-row sequences belong to the prefill kernel, which also
-            // reports malformed cu_seqlens_q
-            if (ce - cb != 1 || cb < 0 || ce > p.total_q) continue;
-        }
         const bool bad = L < 0 || (long long)L > (long long)p.max_blocks_per_seq * p.block_size ||
-                         (p.cu_seqlens_q != nullptr && L < 1);
+                         (p.cu_seqlens_q != nullptr && L < n);
         if (bad) report_error(NPV_DEVERR_CONTEXT_LEN);
-        if (L <= 0 || bad) {
+        if (L < n || bad) {
             uint4 *orow = reinterpret_cast<uint4 *>(p.out + query_row(p, (int32_t)b) * (int64_t)p.num_q_heads * D);
-            for (int i = 0; i < p.num_q_heads * D / 8; ++i) orow[i] = make_uint4(0, 0, 0, 0);
+            for (int i = 0; i < n * p.num_q_heads * D / 8; ++i) orow[i] = make_uint4(0, 0, 0, 0);
             // a fused store still writes this sequence's token
             if (p.key != nullptr) store_token_rows(p, (int32_t)b, 0, p.num_kv_heads, D, 0, 1);
         }
@@ -615,13 +724,16 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const Params p, int h
     grid_dependency_wait();
     if (!work) return;
     const int32_t b = (int32_t)(u / NHG), hg = (int32_t)(u % NHG);
-    uint16_t *orow = p.out + query_row(p, b) * (int64_t)p.num_q_heads * D + (int64_t)hg * HCG * D;
-    for (int idx = threadIdx.x; idx < HCG * D / 4; idx += blockDim.x) {
-        const int h = idx / (D / 4), d4 = (idx % (D / 4)) * 4;
-        float M = p.part_ml[(2 * ca + sa) * HCG + h].x;
+    const int R = g * path_rows(p, b);
+    const int64_t row0 = query_row(p, b);
+    for (int idx = threadIdx.x; idx < HC * R * D / 4; idx += blockDim.x) {
+        const int hl = idx / (R * D / 4), rem = idx % (R * D / 4);
+        const int r = rem / (D / 4), d4 = (rem % (D / 4)) * 4;
+        const long long pr = (long long)hl * RP + r;  // row within a partial slot
+        float M = p.part_ml[(2 * ca + sa) * HC * RP + pr].x;
         for (long long cc = ca + 1; cc <= c; ++cc) {
             if (cc * N / G == (cc + 1) * N / G) continue;  // empty range
-            M = fmaxf(M, p.part_ml[(2 * cc) * HCG + h].x);
+            M = fmaxf(M, p.part_ml[(2 * cc) * HC * RP + pr].x);
         }
         float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f, lsum = 0.f;
         for (long long cc = ca; cc <= c; ++cc) {
@@ -632,9 +744,10 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const Params p, int h
                 if (cc * N / G == (cc + 1) * N / G) continue;
                 slot = 2 * cc;
             }
-            const float2 ml = p.part_ml[slot * HCG + h];
+            const float2 ml = p.part_ml[slot * HC * RP + pr];
+            // a partial whose rows saw only masked keys has m = -inf and weight 0
             const float w = fast_exp2(ml.x - M);
-            const float4 ov = *reinterpret_cast<const float4 *>(p.part_o + (slot * HCG + h) * D + d4);
+            const float4 ov = *reinterpret_cast<const float4 *>(p.part_o + (slot * HC * RP + pr) * D + d4);
             lsum = fmaf(w, ml.y, lsum);
             acc0 = fmaf(w, ov.x, acc0);
             acc1 = fmaf(w, ov.y, acc1);
@@ -643,7 +756,8 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const Params p, int h
         }
         const float inv = 1.0f / lsum;
         uint2 packed = make_uint2(pack_bf16x2(acc0 * inv, acc1 * inv), pack_bf16x2(acc2 * inv, acc3 * inv));
-        *reinterpret_cast<uint2 *>(orow + (int64_t)h * D + d4) = packed;
+        uint16_t *orow = p.out + ((row0 + r / g) * p.num_q_heads + (int64_t)(hg * HC + hl) * g + r % g) * D;
+        *reinterpret_cast<uint2 *>(orow + d4) = packed;
     }
 }
 

@@ -70,13 +70,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 
 // Wait for the phase of `bar` with the given parity to complete.  Returns false
 // (after recording NPV_DEVERR_TIMEOUT) if it does not complete within
-// kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// limit_ns.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+        if ((it & 63u) == 0 && global_timer_ns() - t0 > limit_ns) {
             report_error(NPV_DEVERR_TIMEOUT);
             return false;
         }

@@ -76,6 +76,8 @@ struct DecodeConfig {
     int group = 0;           // g = Hq / Hkv
     int heads_per_cta = 0;   // HC
     int head_groups = 0;     // Hkv / HC
+    int max_rows = 0;        // most query rows of a sequence the kernel serves
+    int rows_per_head = 0;   // partial-slot rows per KV head: g * max_rows
     int stages = 0;
     int grid = 0;
     size_t smem = 0;
@@ -85,13 +87,17 @@ struct DecodeConfig {
 bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
 
 // Largest divisor of Hkv within the kernel's consumer-warp budget (one warp per KV head).
-int pick_heads_per_cta(int num_kv_heads, int g) {
-    for (int hc = npv::decode::max_heads_per_cta(g); hc >= 1; --hc)
+int pick_heads_per_cta(int num_kv_heads) {
+    for (int hc = npv::decode::kMaxConsumerWarps; hc >= 1; --hc)
         if (num_kv_heads % hc == 0) return hc;
     return 1;
 }
 
-npv_status decode_config(int num_q_heads, int num_kv_heads, int head_dim, DecodeConfig *cfg) {
+// multi_row: the decode kernel also serves sequences of up to 16 / g query rows
+// (the rows of a prefill call that fit its two 8-column MMA tiles per KV head);
+// the workspace is sized for that.
+npv_status decode_config(int num_q_heads, int num_kv_heads, int head_dim, DecodeConfig *cfg,
+                         bool multi_row = false) {
     if (num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return NPV_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return NPV_ERR_UNSUPPORTED;
     const int g = num_q_heads / num_kv_heads;
@@ -99,28 +105,29 @@ npv_status decode_config(int num_q_heads, int num_kv_heads, int head_dim, Decode
     const DeviceInfo *dev = current_device();
     if (!dev) return NPV_ERR_CUDA;
     cfg->group = g;
-    cfg->heads_per_cta = pick_heads_per_cta(num_kv_heads, g);
+    cfg->heads_per_cta = pick_heads_per_cta(num_kv_heads);
     cfg->head_groups = num_kv_heads / cfg->heads_per_cta;
+    cfg->max_rows = multi_row ? npv::decode::kTileRows / g : 1;
+    cfg->rows_per_head = g * cfg->max_rows;
     const int hc = cfg->heads_per_cta;
     const size_t stage_bytes = 2ull * npv::decode::kChunk * hc * head_dim * 2;
     int stages = (int)(npv::decode::kStageBudgetBytes / stage_bytes);
     if (stages > npv::decode::kMaxStages) stages = npv::decode::kMaxStages;
     if (stages < 2) stages = 2;
     cfg->stages = stages;
-    const size_t pbuf = align_up((size_t)hc * npv::decode::kChunk * g * 4, 1024);
-    cfg->smem = npv::decode::kHeaderBytes + pbuf + stages * stage_bytes;
+    cfg->smem = npv::decode::kHeaderBytes + stages * stage_bytes;
     if ((int)cfg->smem > dev->max_smem_optin) return NPV_ERR_UNSUPPORTED;
     cfg->grid = dev->sm_count;
-    const size_t hcg = (size_t)hc * g;
-    cfg->ws_ml = align_up((size_t)cfg->grid * 2 * hcg * sizeof(float2), 256);
-    cfg->ws_o = align_up((size_t)cfg->grid * 2 * hcg * head_dim * sizeof(float), 256);
+    const size_t rows = (size_t)hc * cfg->rows_per_head;
+    cfg->ws_ml = align_up((size_t)cfg->grid * 2 * rows * sizeof(float2), 256);
+    cfg->ws_o = align_up((size_t)cfg->grid * 2 * rows * head_dim * sizeof(float), 256);
     cfg->ws_total = cfg->ws_ml + cfg->ws_o;
     return NPV_OK;
 }
 
-template <int D, int G>
+template <int D, int G, int NR>
 cudaError_t launch_decode_split(const npv::decode::Params &p, const DecodeConfig &cfg, cudaStream_t stream) {
-    auto kernel = npv::decode::decode_split_kernel<D, G>;
+    auto kernel = npv::decode::decode_split_kernel<D, G, NR>;
     static int configured_smem[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -134,8 +141,11 @@ cudaError_t launch_decode_split(const npv::decode::Params &p, const DecodeConfig
 
 cudaError_t dispatch_decode_split(int D, const npv::decode::Params &p, const DecodeConfig &cfg,
                                   cudaStream_t stream) {
-#define NPV_DECODE_CASE(DD, GG) \
-    if (D == DD && cfg.group == GG) return launch_decode_split<DD, GG>(p, cfg, stream);
+    const int nr = cfg.rows_per_head > 8 ? 2 : 1;
+#define NPV_DECODE_CASE(DD, GG)                                                         \
+    if (D == DD && cfg.group == GG)                                                     \
+        return nr == 1 ? launch_decode_split<DD, GG, 1>(p, cfg, stream)                 \
+                       : launch_decode_split<DD, GG, 2>(p, cfg, stream);
     NPV_DECODE_CASE(128, 1)
     NPV_DECODE_CASE(128, 2)
     NPV_DECODE_CASE(128, 4)
@@ -182,6 +192,8 @@ npv_status run_decode(void *out, const void *q, int64_t q_row_stride, const int3
     p.block_size = block_size;
     p.heads_per_cta = cfg.heads_per_cta;
     p.num_head_groups = cfg.head_groups;
+    p.max_rows = cfg.max_rows;
+    p.rows_per_head = cfg.rows_per_head;
     p.num_stages = cfg.stages;
     const float s = scale > 0.f ? scale : (float)(1.0 / std::sqrt((double)head_dim));
     p.scale_log2 = s * 1.4426950408889634f;
@@ -247,7 +259,7 @@ struct PrefillConfig {
 npv_status prefill_config(int32_t num_seqs, int32_t total_q, int num_q_heads, int num_kv_heads, int head_dim,
                           PrefillConfig *cfg) {
     if (num_seqs < 0 || total_q < 0) return NPV_ERR_INVALID_ARG;
-    npv_status st = decode_config(num_q_heads, num_kv_heads, head_dim, &cfg->decode);
+    npv_status st = decode_config(num_q_heads, num_kv_heads, head_dim, &cfg->decode, true);
     if (st != NPV_OK) return st;
     const DeviceInfo *dev = current_device();
     if (!dev) return NPV_ERR_CUDA;
@@ -498,12 +510,27 @@ npv_status npv_paged_prefill_attention(void *out, const void *q, const int32_t *
     p.ml_x = reinterpret_cast<float2 *>(ws + cfg.decode.ws_total + 256 + cfg.ws_pairs);
     p.max_pairs = cfg.max_pairs;
 
+    // The decode kernel takes the sequences whose g * n_b rows fit its MMA
+    // columns: one 8-column tile when max_seqlen_q says that suffices (fewer
+    // registers), else two.  The hint only moves sequences between the two
+    // kernels, which both routes use alike, so a wrong hint costs speed, never
+    // correctness.
+    if ((int64_t)max_seqlen_q * G <= 8) {
+        cfg.decode.max_rows = 8 / G;
+        cfg.decode.rows_per_head = 8;
+    }
+    p.decode_rows_max = cfg.decode.max_rows;
     cudaError_t e = dispatch_prefill(D, G, p, qmap, kmap, vmap, cfg, s);
     if (e != cudaSuccess) return NPV_ERR_CUDA;
-    // rows of sequences with exactly one query row: split-KV decode
+    // sequences of 1 .. 16 / g query rows: the split-KV decode kernel
     return run_decode(out, q, (int64_t)num_q_heads * head_dim, cu_seqlens_q, total_q, k_cache, v_cache,
                       block_tables, max_blocks_per_seq, context_lens, num_seqs, num_q_heads, num_kv_heads,
                       head_dim, num_blocks, block_size, scale, workspace, cfg.decode, s);
+}
+
+npv_status npv_debug_inject_decode_timeout(int enable) {
+    const unsigned int v = enable ? 1u : 0u;
+    return cuda_status(cudaMemcpyToSymbol(npv::decode::g_debug_timeout, &v, sizeof(v)));
 }
 
 npv_status npv_check_device_errors(npv_stream_t stream, uint32_t *bits_out) {

@@ -3,11 +3,12 @@
 //
 // What it computes ("nano-vllm" README, Features: Chunked Prefill and Prefix
 // Caching, Tutorial Mode chapter 3 on the causal mask; "Nano-vLLM Architecture
-// and Performance", Key Features 1): for sequence b with n_b >= 2 new rows that
+// and Performance", Key Features 1): for sequence b with n_b new rows that
 // are already stored at positions L_b - n_b .. L_b - 1, row i attends to keys
 // 0 .. L_b - n_b + i of the sequence's paged K/V, query head h reading KV head
-// h / g, scale 1/sqrt(D) by default.  Rows of sequences with n_b == 1 go to
-// the split-KV decode kernel in the same call.
+// h / g, scale 1/sqrt(D) by default.  This kernel takes the sequences with
+// n_b > 16 / g; shorter ones (decode rows, speculative-decode verification)
+// go to the split-KV decode kernel in the same call.
 //
 // How (B200 design):
 //   * Work item = (sequence, KV head, tile of 128 MMA rows).  The 128 rows pack
@@ -60,6 +61,7 @@ constexpr int kTileM = 128;   // query rows per item (MMA M)
 constexpr int kTileN = 128;   // keys per KV tile (MMA N of S, K of P.V)
 constexpr int kKStages = 3;   // K ring depth (a K stage is free once S = Q K^T is done)
 constexpr int kVStages = 3;   // V ring depth (a V stage is free once O += P V is done)
+constexpr int kMaxRing = kKStages > kVStages ? kKStages : kVStages;
 constexpr int kThreads = 384;  // MMA, K producer, V producer, Q producer, 8 softmax warps
 constexpr int kMmaWarp = 0;
 constexpr int kKProducerWarp = 1;
@@ -90,6 +92,7 @@ struct Params {
     int32_t *plan_count;  // [1]: number of (sequence, row-tile) pairs
     int2 *plan_pairs;     // [max_pairs]: (sequence, row tile), longest first
     int32_t max_pairs;
+    int32_t decode_rows_max;  // sequences with at most this many query rows run on the decode kernel
     float2 *ml_x;         // [grid][2 item parities][2 warpgroups][128 rows]: (m, l) exchange
 };
 
@@ -143,7 +146,8 @@ __device__ __forceinline__ long long item_index(long long r) {
     return r * G + ((r & 1) ? (G - 1 - blockIdx.x) : blockIdx.x);
 }
 
-// A sequence runs on the tensor-core path when it has >= 2 valid query rows.
+// A sequence runs on this kernel when it has more query rows than the decode
+// kernel's warp-level tile takes (n_b > decode_rows_max = 16 / g).
 __device__ __forceinline__ bool prefill_seq(const Params &p, int32_t b, int32_t *n_out, bool *bad) {
     const int32_t cb = __ldg(p.cu_seqlens_q + b), ce = __ldg(p.cu_seqlens_q + b + 1);
     *bad = false;
@@ -154,7 +158,7 @@ __device__ __forceinline__ bool prefill_seq(const Params &p, int32_t b, int32_t 
     }
     const int32_t n = ce - cb;
     *n_out = n;
-    if (n < 2) return false;
+    if (n <= p.decode_rows_max) return false;
     const int32_t L = __ldg(p.context_lens + b);
     if (L < n || (long long)L > (long long)p.max_blocks_per_seq * p.block_size) {
         *bad = true;
@@ -314,10 +318,13 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, vo
     return __all_sync(0xffffffffu, ok);
 }
 
-#define NPV_WAIT(bar, parity)                                   \
-    do {                                                        \
-        if (!wait_or_abort((bar), (parity), abort_flag)) goto finish; \
+// A wait that gives up leaves the warp's loops for `label`, where the warp
+// first settles what it has in flight, then meets the others at `finish`.
+#define NPV_WAIT_OR(bar, parity, label)                               \
+    do {                                                              \
+        if (!wait_or_abort((bar), (parity), abort_flag)) goto label; \
     } while (0)
+#define NPV_WAIT(bar, parity) NPV_WAIT_OR(bar, parity, finish)
 
 __device__ __forceinline__ void setmaxnreg_dec56() { asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory"); }
 __device__ __forceinline__ void setmaxnreg_inc224() { asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory"); }
@@ -344,6 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *ml_full = o_free + 1;         // per-row (m, l) of both warpgroups exchanged (8 softmax warps)
     uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(ml_full + 1);
     int *abort_flag = reinterpret_cast<int *>(ml_full + 2);
+    uint64_t *mma_drain = ml_full + 3;      // every tcgen05.mma issued so far is done (exit path)
     float2 *xml = p.ml_x + (size_t)blockIdx.x * (2 * 2 * kTileM);  // this CTA's exchange slots
     uint8_t *sQ = smem + L::q;
     uint8_t *sK = smem + L::k;
@@ -371,6 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(o_full, 1);
         mbar_init(o_free, kSoftmaxWarps);
         mbar_init(ml_full, kSoftmaxWarps);
+        mbar_init(mma_drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -396,11 +405,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ============================ Q tiles (TMA) ============================
         setmaxnreg_dec56();
         uint32_t item_iter = 0;
+        bool q_filled = false;  // the last Q tile's copy, waited for before the CTA ends
+        uint32_t q_parity = 0;
         for (long long r = 0; r < rounds; ++r, ++item_iter) {
             const long long idx = item_index(r);
             if (idx >= n_items) break;
             const Item it = load_item<G>(p, idx);
-            NPV_WAIT(q_empty, (item_iter & 1) ^ 1);  // the previous item's S products are done
+            NPV_WAIT_OR(q_empty, (item_iter & 1) ^ 1, q_exit);  // the previous item's S products are done
+            q_filled = true;
+            q_parity = item_iter & 1;
             if (lane == 0) {
                 mbar_arrive_expect_tx(q_full, (uint32_t)(kTileM * D * 2));
                 // rows (position, head) of the tile: box {64 elements, G heads, 128 / G positions}
@@ -409,6 +422,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncwarp();
         }
+    q_exit:
+        // the shared memory of a CTA must outlive every copy into it, also when a
+        // wait gave up and the loop was left early (bounded: a copy always lands)
+        if (q_filled) mbar_wait(q_full, q_parity);
     } else if (warp == kKProducerWarp || warp == kVProducerWarp) {
         // ============================ K / V tiles (TMA) ============================
         setmaxnreg_dec56();
@@ -420,6 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const CUtensorMap *map = is_k ? &kmap : &vmap;
         uint32_t kv_iter = 0;
         const int BS = p.block_size;
+        uint32_t filled = 0, filled_parity = 0;  // per stage: ever filled, parity of its last fill
         for (long long r = 0; r < rounds; ++r) {
             const long long idx = item_index(r);
             if (idx >= n_items) break;
@@ -428,9 +446,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             int win = -1, win_val = -1;
             for (int t = 0; t < it.ntiles; ++t, ++kv_iter) {
                 const int s = (int)(kv_iter % nstages);
-                NPV_WAIT(&empty[s], ((kv_iter / nstages) & 1) ^ 1);
+                NPV_WAIT_OR(&empty[s], ((kv_iter / nstages) & 1) ^ 1, kv_exit);
                 int blk_of_box[8];
                 const int nload = tile_boxes(p, it, bt_row, t, lane, win, win_val, blk_of_box);
+                filled |= 1u << s;
+                filled_parity = (filled_parity & ~(1u << s)) | (((kv_iter / nstages) & 1u) << s);
                 if (lane == 0) {
                     const uint32_t bytes = (uint32_t)(nload * p.box_tokens * 128 * kDBlocks);
                     uint8_t *dst = ring + s * L::kKV;
@@ -451,6 +471,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
             }
         }
+    kv_exit:
+        for (int st = 0; st < nstages; ++st)
+            if (filled & (1u << st)) mbar_wait(&full[st], (filled_parity >> st) & 1u);
     } else if (warp == kMmaWarp) {
         // ============================ MMA issuer ============================
         setmaxnreg_dec56();
@@ -467,16 +490,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const long long idx = item_index(r);
             if (idx >= n_items) break;
             const Item it = load_item<G>(p, idx);
-            NPV_WAIT(q_full, item_iter & 1);
+            NPV_WAIT_OR(q_full, item_iter & 1, mma_exit);
             for (int t = -2; t < it.ntiles; ++t) {
                 if (t >= 0) {
                     // ---- O_j (+)= P_t V_t, j = T & 1 (P from tensor memory, over S_t)
                     const uint32_t T = kv_iter + t;
                     const int j = (int)(T & 1);
                     const int vs = (int)(T % kVStages);
-                    NPV_WAIT(&p_full[j], (T >> 1) & 1);
-                    NPV_WAIT(&v_full[vs], (T / kVStages) & 1);
-                    if (t == 0) NPV_WAIT(o_free, (item_iter & 1) ^ 1);
+                    NPV_WAIT_OR(&p_full[j], (T >> 1) & 1, mma_exit);
+                    NPV_WAIT_OR(&v_full[vs], (T / kVStages) & 1, mma_exit);
+                    if (t == 0) NPV_WAIT_OR(o_free, (item_iter & 1) ^ 1, mma_exit);
                     const int valid = min(kTileN, it.kv_end - t * kTileN);
                     const int ksteps = (valid + 15) / 16;
                     if (valid < ksteps * 16) {
@@ -511,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // ---- S_ts = Q K_ts^T into buffer T & 1
                     const uint32_t T = kv_iter + ts;
                     const int ks = (int)(T % kKStages);
-                    NPV_WAIT(&k_full[ks], (T / kKStages) & 1);
+                    NPV_WAIT_OR(&k_full[ks], (T / kKStages) & 1, mma_exit);
                     tc::fence_after_sync();
                     if (lane == 0) {
                         const uint32_t d = tmem + (T & 1) * kTileN;
@@ -531,6 +554,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             kv_iter += it.ntiles;
             ++item_iter;
         }
+    mma_exit:
+        // tensor-core operations still reading shared memory or writing tensor memory
+        if (lane == 0) {
+            tc::mma_commit(mma_drain);
+            mbar_wait(mma_drain, 0);
+        }
+        __syncwarp();
     } else if (warp >= kFirstSoftmaxWarp) {
         // ==== softmax: warpgroup j (warps 4 + 4 j .. 7 + 4 j) takes the KV tiles T with T % 2 == j ====
         // Registers: the launch gives every thread 168; the first warpgroup (MMA,
@@ -699,6 +729,7 @@ finish:
 }
 
 #undef NPV_WAIT
+#undef NPV_WAIT_OR
 
 }  // namespace prefill
 }  // namespace npv

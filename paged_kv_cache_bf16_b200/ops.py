@@ -74,6 +74,8 @@ def lib() -> C.CDLL:
     l.npv_paged_prefill_attention.restype = C.c_int
     l.npv_check_device_errors.argtypes = [p, C.POINTER(C.c_uint32)]
     l.npv_check_device_errors.restype = C.c_int
+    l.npv_debug_inject_decode_timeout.argtypes = [C.c_int]
+    l.npv_debug_inject_decode_timeout.restype = C.c_int
     _lib = l
     return l
 
@@ -232,6 +234,12 @@ def check_device_errors(stream=None) -> int:
     if st != NPV_OK:
         raise NpvError(st, "npv_check_device_errors", bits.value)
     return bits.value
+
+
+def inject_decode_timeout(enable: bool) -> None:
+    """Failure-detection test hook: make the decode kernel's bounded pipeline wait give up
+    (see npv_debug_inject_decode_timeout in include/npv.h)."""
+    _check(lib().npv_debug_inject_decode_timeout(1 if enable else 0), "npv_debug_inject_decode_timeout")
 
 
 def default_scale(head_dim: int) -> float:
