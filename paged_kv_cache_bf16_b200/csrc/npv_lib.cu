@@ -252,7 +252,7 @@ struct PrefillConfig {
     int32_t max_pairs = 0;
     int grid = 0;
     size_t smem = 0;
-    size_t ws_pairs = 0, ws_mlx = 0;
+    size_t ws_pairs = 0;
     size_t ws_total = 0;
 };
 
@@ -271,9 +271,7 @@ npv_status prefill_config(int32_t num_seqs, int32_t total_q, int num_q_heads, in
     cfg->smem = (head_dim == 128 ? npv::prefill::Smem<128>::total : npv::prefill::Smem<64>::total) + 1024;
     if ((int)cfg->smem > dev->max_smem_optin) return NPV_ERR_UNSUPPORTED;
     cfg->ws_pairs = align_up((size_t)pairs * sizeof(int2), 256);
-    // per CTA: (m, l) exchange slots of the two softmax warpgroups, by item parity
-    cfg->ws_mlx = (size_t)cfg->grid * 2 * 2 * npv::prefill::kTileM * sizeof(float2);
-    cfg->ws_total = cfg->decode.ws_total + 256 + cfg->ws_pairs + cfg->ws_mlx;
+    cfg->ws_total = cfg->decode.ws_total + 256 + cfg->ws_pairs;
     return NPV_OK;
 }
 
@@ -507,7 +505,6 @@ npv_status npv_paged_prefill_attention(void *out, const void *q, const int32_t *
     char *ws = static_cast<char *>(workspace);
     p.plan_count = reinterpret_cast<int32_t *>(ws + cfg.decode.ws_total);
     p.plan_pairs = reinterpret_cast<int2 *>(ws + cfg.decode.ws_total + 256);
-    p.ml_x = reinterpret_cast<float2 *>(ws + cfg.decode.ws_total + 256 + cfg.ws_pairs);
     p.max_pairs = cfg.max_pairs;
 
     // The decode kernel takes the sequences whose g * n_b rows fit its MMA

@@ -57,12 +57,11 @@
 namespace npv {
 namespace prefill {
 
-constexpr int kTileM = 128;   // query rows per item (MMA M)
+constexpr int kTileM = 128;   // query rows per Q tile (MMA M); an item holds two Q tiles
 constexpr int kTileN = 128;   // keys per KV tile (MMA N of S, K of P.V)
-constexpr int kKStages = 3;   // K ring depth (a K stage is free once S = Q K^T is done)
-constexpr int kVStages = 3;   // V ring depth (a V stage is free once O += P V is done)
-constexpr int kMaxRing = kKStages > kVStages ? kKStages : kVStages;
-constexpr int kThreads = 384;  // MMA, K producer, V producer, Q producer, 8 softmax warps
+constexpr int kKStages = 2;   // K ring depth (a K stage is free once both S = Q K^T products are done)
+constexpr int kVStages = 3;   // V ring depth (a V stage is free once both O += P V products are done)
+constexpr int kThreads = 384;  // MMA, K producer, V producer, Q producer, 2 softmax warpgroups
 constexpr int kMmaWarp = 0;
 constexpr int kKProducerWarp = 1;
 constexpr int kVProducerWarp = 2;
@@ -70,7 +69,7 @@ constexpr int kQProducerWarp = 3;
 constexpr int kFirstSoftmaxWarp = 4;
 constexpr int kSoftmaxWarps = 8;
 constexpr int kTmemCols = 512;
-constexpr int kTmemO = 2 * kTileN;  // O_0 at [256, 256 + D), O_1 at [256 + D, 256 + 2 D)
+constexpr int kTmemO = 2 * kTileN;  // S_A, S_B at [0, 256); O_A at [256, 256 + D), O_B at [384, 384 + D)
 constexpr int kBuckets = 4096;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -93,32 +92,35 @@ struct Params {
     int2 *plan_pairs;     // [max_pairs]: (sequence, row tile), longest first
     int32_t max_pairs;
     int32_t decode_rows_max;  // sequences with at most this many query rows run on the decode kernel
-    float2 *ml_x;         // [grid][2 item parities][2 warpgroups][128 rows]: (m, l) exchange
 };
 
-// Shared-memory layout (bytes from a 1024-aligned base): barriers, then the Q
-// tile and the K and V rings (3 + 3 stages of 32 KB at D = 128: 225 KB in all,
-// which is why the warpgroups' per-item (m, l) exchange goes through a
-// CTA-private slot in global memory instead).
+// Shared-memory layout (bytes from a 1024-aligned base): barriers, then the two
+// Q tiles of an item and the K and V rings (2 x 32 + 2 + 3 stages of 32 KB at
+// D = 128: 225 KB in all).
 template <int D>
 struct Smem {
     static constexpr int kHeader = 1024;
     static constexpr int kKV = kTileN * D * 2;
+    static constexpr int kQ = kTileM * D * 2;
     static constexpr int q = kHeader;
-    static constexpr int k = q + kTileM * D * 2;
+    static constexpr int k = q + 2 * kQ;
     static constexpr int v = k + kKStages * kKV;
     static constexpr int total = v + kVStages * kKV;
 };
 
-// Per-item quantities every warp role derives the same way.
+// Per-item quantities every warp role derives the same way.  An item is a
+// (sequence, KV head, pair of Q tiles): Q tile A holds positions p0 .. p0 + ppt - 1,
+// Q tile B the next ppt positions (ppt = 128 / g positions x g heads = 128 MMA
+// rows each); both read the same K/V tiles, loaded once.
 struct Item {
     int32_t b, qt, h;
     int32_t row0;    // first packed query row of the sequence
     int32_t n;       // query rows of the sequence
     int32_t L;       // context length (new rows included)
-    int32_t p0;      // first position of this row tile (relative to the new rows)
-    int32_t npos;    // positions in this tile
-    int32_t kv_end;  // keys the tile needs: [0, kv_end)
+    int32_t p0;      // first position of Q tile A (relative to the new rows)
+    int32_t npos_a;  // positions in Q tile A
+    int32_t npos_b;  // positions in Q tile B (0 .. ppt)
+    int32_t kv_end;  // keys the item needs: [0, kv_end)
     int32_t ntiles;  // 128-key tiles
 };
 
@@ -133,9 +135,10 @@ __device__ __forceinline__ Item load_item(const Params &p, long long idx) {
     it.n = __ldg(p.cu_seqlens_q + it.b + 1) - it.row0;
     it.L = __ldg(p.context_lens + it.b);
     constexpr int ppt = kTileM / G;
-    it.p0 = it.qt * ppt;
-    it.npos = min(ppt, it.n - it.p0);
-    it.kv_end = min(it.L, it.L - it.n + it.p0 + it.npos);
+    it.p0 = it.qt * 2 * ppt;
+    it.npos_a = min(ppt, it.n - it.p0);
+    it.npos_b = max(0, min(ppt, it.n - it.p0 - ppt));
+    it.kv_end = min(it.L, it.L - it.n + it.p0 + it.npos_a + it.npos_b);
     it.ntiles = (it.kv_end + kTileN - 1) / kTileN;
     return it;
 }
@@ -168,14 +171,14 @@ __device__ __forceinline__ bool prefill_seq(const Params &p, int32_t b, int32_t 
 }
 
 // ---------------------------------------------------------------------------
-// plan: list the (sequence, row tile) pairs, longest KV range first
+// plan: list the (sequence, pair of Q tiles) items, longest KV range first
 // ---------------------------------------------------------------------------
 template <int G>
 __global__ void __launch_bounds__(1024) prefill_plan_kernel(const Params p, int head_dim) {
     __shared__ int hist[kBuckets];
     __shared__ long long scratch[40];
     grid_dependency_wait();
-    constexpr int ppt = kTileM / G;
+    constexpr int ppt = 2 * (kTileM / G);  // positions per item (two Q tiles)
     const int tid = threadIdx.x;
     for (int i = tid; i < kBuckets; i += blockDim.x) hist[i] = 0;
     const int per = (p.num_seqs + blockDim.x - 1) / blockDim.x;
@@ -338,21 +341,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // 128-byte-swizzled tiles need 1024-byte-aligned shared addresses
     uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
-    uint64_t *q_full = bars + 0;   // Q tile landed (TMA)
-    uint64_t *q_empty = bars + 1;  // the item's last S product is done
+    uint64_t *q_full = bars + 0;   // both Q tiles landed (TMA)
+    uint64_t *q_empty = bars + 1;  // the item's last S products are done
     uint64_t *k_full = bars + 2;   // [kKStages]
-    uint64_t *k_empty = bars + 2 + kKStages;
-    uint64_t *v_full = bars + 2 + 2 * kKStages;  // [kVStages]
+    uint64_t *k_empty = k_full + kKStages;
+    uint64_t *v_full = k_empty + kKStages;  // [kVStages]
     uint64_t *v_empty = v_full + kVStages;
-    uint64_t *s_full = v_empty + kVStages;  // [2]: S tile in buffer j is ready
-    uint64_t *p_full = s_full + 2;          // [2]: P written over buffer j (4 warps of warpgroup j)
-    uint64_t *o_full = p_full + 2;          // the item's last P.V product is done
-    uint64_t *o_free = o_full + 1;          // both O accumulators read out (8 softmax warps)
-    uint64_t *ml_full = o_free + 1;         // per-row (m, l) of both warpgroups exchanged (8 softmax warps)
-    uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(ml_full + 1);
-    int *abort_flag = reinterpret_cast<int *>(ml_full + 2);
-    uint64_t *mma_drain = ml_full + 3;      // every tcgen05.mma issued so far is done (exit path)
-    float2 *xml = p.ml_x + (size_t)blockIdx.x * (2 * 2 * kTileM);  // this CTA's exchange slots
+    uint64_t *s_full = v_empty + kVStages;  // [2]: S of Q tile j (A = 0, B = 1) is ready
+    uint64_t *p_full = s_full + 2;          // [2]: P of Q tile j written over its S (4 warps)
+    uint64_t *o_full = p_full + 2;          // [2]: the item's last P.V product of Q tile j is done
+    uint64_t *o_free = o_full + 2;          // both O accumulators read out (8 softmax warps)
+    uint64_t *mma_drain = o_free + 1;       // every tcgen05.mma issued so far is done (exit path)
+    uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(mma_drain + 1);
+    int *abort_flag = reinterpret_cast<int *>(mma_drain + 2);
     uint8_t *sQ = smem + L::q;
     uint8_t *sK = smem + L::k;
     uint8_t *sV = smem + L::v;
@@ -360,6 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int kDBlocks = D / 64;           // 64-element (128-byte) column blocks
     constexpr int kBlockBytes = kTileN * 128;  // one column block of a 128-row Q, K or V tile
+    constexpr int ppt = kTileM / G;            // positions per Q tile
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -375,10 +377,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 2; ++j) {
             mbar_init(&s_full[j], 1);
             mbar_init(&p_full[j], kSoftmaxWarps / 2);
+            mbar_init(&o_full[j], 1);
         }
-        mbar_init(o_full, 1);
         mbar_init(o_free, kSoftmaxWarps);
-        mbar_init(ml_full, kSoftmaxWarps);
         mbar_init(mma_drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -405,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ============================ Q tiles (TMA) ============================
         setmaxnreg_dec56();
         uint32_t item_iter = 0;
-        bool q_filled = false;  // the last Q tile's copy, waited for before the CTA ends
+        bool q_filled = false;  // the last Q tiles' copy, waited for before the CTA ends
         uint32_t q_parity = 0;
         for (long long r = 0; r < rounds; ++r, ++item_iter) {
             const long long idx = item_index(r);
@@ -415,10 +416,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             q_filled = true;
             q_parity = item_iter & 1;
             if (lane == 0) {
-                mbar_arrive_expect_tx(q_full, (uint32_t)(kTileM * D * 2));
-                // rows (position, head) of the tile: box {64 elements, G heads, 128 / G positions}
-                for (int db = 0; db < kDBlocks; ++db)
-                    tc::tma_load_3d(sQ + db * kBlockBytes, &qmap, db * 64, it.h * G, it.row0 + it.p0, q_full);
+                mbar_arrive_expect_tx(q_full, (uint32_t)(2 * kTileM * D * 2));
+                // rows (position, head) of each tile: box {64 elements, G heads, 128 / G positions};
+                // tile B's rows past the last query row read the map's zero fill
+                for (int j = 0; j < 2; ++j)
+                    for (int db = 0; db < kDBlocks; ++db)
+                        tc::tma_load_3d(sQ + j * L::kQ + db * kBlockBytes, &qmap, db * 64, it.h * G,
+                                        it.row0 + it.p0 + j * ppt, q_full);
             }
             __syncwarp();
         }
@@ -477,9 +481,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kMmaWarp) {
         // ============================ MMA issuer ============================
         setmaxnreg_dec56();
-        // Order within an item: S_0, S_1, then PV_t followed by S_{t+2}.  S_{t+2}
-        // overwrites the buffer that P_t occupies, which PV_t (issued before it
-        // by this thread) reads; tcgen05.mma ops of one thread run in order.
+        // Per KV tile t of an item, in this order: PV_A(t), S_A(t+1), PV_B(t),
+        // S_B(t+1).  S_j(t+1) overwrites the columns P_j(t) occupies, which
+        // PV_j(t), issued before it by this thread, reads (tcgen05.mma ops of one
+        // thread run in order).  While softmax warpgroup A works on tile t the
+        // tensor pipe runs B's products, and the other way round.
         constexpr uint32_t idesc_s = tc::idesc_bf16_f32(kTileM, kTileN, 0, 0);
         constexpr uint32_t idesc_o = tc::idesc_bf16_f32(kTileM, D, 0, 1);
         const uint64_t qdesc = tc::smem_desc_sw128(smem_addr(sQ), 16, 1024);
@@ -491,64 +497,71 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (idx >= n_items) break;
             const Item it = load_item<G>(p, idx);
             NPV_WAIT_OR(q_full, item_iter & 1, mma_exit);
-            for (int t = -2; t < it.ntiles; ++t) {
-                if (t >= 0) {
-                    // ---- O_j (+)= P_t V_t, j = T & 1 (P from tensor memory, over S_t)
-                    const uint32_t T = kv_iter + t;
-                    const int j = (int)(T & 1);
-                    const int vs = (int)(T % kVStages);
-                    NPV_WAIT_OR(&p_full[j], (T >> 1) & 1, mma_exit);
-                    NPV_WAIT_OR(&v_full[vs], (T / kVStages) & 1, mma_exit);
-                    if (t == 0) NPV_WAIT_OR(o_free, (item_iter & 1) ^ 1, mma_exit);
-                    const int valid = min(kTileN, it.kv_end - t * kTileN);
-                    const int ksteps = (valid + 15) / 16;
-                    if (valid < ksteps * 16) {
-                        // zero the V rows of the last K step that lie past the context
-                        uint8_t *vsm = sV + vs * L::kKV;
-                        const int nrows = ksteps * 16 - valid;
-                        for (int e = lane; e < nrows * 8 * kDBlocks; e += 32) {
-                            const int db = e / (nrows * 8);
-                            const int rr = valid + (e % (nrows * 8)) / 8;
-                            const int ch = e % 8;
-                            *reinterpret_cast<uint4 *>(vsm + db * kBlockBytes + rr * 128 + ch * 16) =
-                                make_uint4(0, 0, 0, 0);
+            for (int t = -1; t < it.ntiles; ++t) {
+                const int tn = t + 1;  // the tile whose S products follow
+                const uint32_t Tn = kv_iter + tn;
+                const int ks = (int)(Tn % kKStages);
+                for (int j = 0; j < 2; ++j) {
+                    if (t >= 0) {
+                        // ---- O_j (+)= P_j(t) V_t (P from tensor memory, over S_j)
+                        const uint32_t T = kv_iter + t;
+                        const int vs = (int)(T % kVStages);
+                        NPV_WAIT_OR(&p_full[j], T & 1, mma_exit);
+                        if (j == 0) {
+                            NPV_WAIT_OR(&v_full[vs], (T / kVStages) & 1, mma_exit);
+                            if (t == 0) NPV_WAIT_OR(o_free, (item_iter & 1) ^ 1, mma_exit);
                         }
-                        tc::fence_proxy_async_smem();
+                        const int valid = min(kTileN, it.kv_end - t * kTileN);
+                        const int ksteps = (valid + 15) / 16;
+                        if (j == 0 && valid < ksteps * 16) {
+                            // zero the V rows of the last K step that lie past the context
+                            uint8_t *vsm = sV + vs * L::kKV;
+                            const int nrows = ksteps * 16 - valid;
+                            for (int e = lane; e < nrows * 8 * kDBlocks; e += 32) {
+                                const int db = e / (nrows * 8);
+                                const int rr = valid + (e % (nrows * 8)) / 8;
+                                const int ch = e % 8;
+                                *reinterpret_cast<uint4 *>(vsm + db * kBlockBytes + rr * 128 + ch * 16) =
+                                    make_uint4(0, 0, 0, 0);
+                            }
+                            tc::fence_proxy_async_smem();
+                            __syncwarp();
+                        }
+                        tc::fence_after_sync();
+                        if (lane == 0) {
+                            const uint32_t d = tmem + kTmemO + j * 128;
+                            const uint32_t a = tmem + j * kTileN;
+                            const uint64_t vd = vdesc + (uint64_t)((vs * L::kKV) >> 4);
+#pragma unroll
+                            for (int k = 0; k < kTileN / 16; ++k)
+                                if (k < ksteps)
+                                    tc::mma_bf16_ts(d, a + k * 8, vd + (uint64_t)(k * 128), idesc_o, t > 0 || k > 0);
+                            if (j == 1) tc::mma_commit(&v_empty[vs]);
+                            if (t == it.ntiles - 1) tc::mma_commit(&o_full[j]);
+                        }
                         __syncwarp();
                     }
-                    tc::fence_after_sync();
-                    if (lane == 0) {
-                        const uint32_t d = tmem + kTmemO + j * D;
-                        const uint32_t a = tmem + j * kTileN;
-                        const uint64_t vd = vdesc + (uint64_t)((vs * L::kKV) >> 4);
+                    if (tn < it.ntiles) {
+                        // ---- S_j(tn) = Q_j K_tn^T into S_j's columns
+                        if (j == 0) NPV_WAIT_OR(&k_full[ks], (Tn / kKStages) & 1, mma_exit);
+                        tc::fence_after_sync();
+                        if (lane == 0) {
+                            const uint32_t d = tmem + j * kTileN;
+                            const uint64_t qd = qdesc + (uint64_t)((j * L::kQ) >> 4);
+                            const uint64_t kd = kdesc + (uint64_t)((ks * L::kKV) >> 4);
 #pragma unroll
-                        for (int k = 0; k < kTileN / 16; ++k)
-                            if (k < ksteps) tc::mma_bf16_ts(d, a + k * 8, vd + (uint64_t)(k * 128), idesc_o, t >= 2 || k > 0);
-                        tc::mma_commit(&v_empty[vs]);
-                        if (t == it.ntiles - 1) tc::mma_commit(o_full);
-                    }
-                    __syncwarp();
-                }
-                const int ts = t + 2;
-                if (ts < it.ntiles) {
-                    // ---- S_ts = Q K_ts^T into buffer T & 1
-                    const uint32_t T = kv_iter + ts;
-                    const int ks = (int)(T % kKStages);
-                    NPV_WAIT_OR(&k_full[ks], (T / kKStages) & 1, mma_exit);
-                    tc::fence_after_sync();
-                    if (lane == 0) {
-                        const uint32_t d = tmem + (T & 1) * kTileN;
-                        const uint64_t kd = kdesc + (uint64_t)((ks * L::kKV) >> 4);
-#pragma unroll
-                        for (int k = 0; k < D / 16; ++k) {
-                            const uint64_t off = (uint64_t)(((k >> 2) * kBlockBytes + (k & 3) * 32) >> 4);
-                            tc::mma_bf16_ss(d, qdesc + off, kd + off, idesc_s, k > 0);
+                            for (int k = 0; k < D / 16; ++k) {
+                                const uint64_t off = (uint64_t)(((k >> 2) * kBlockBytes + (k & 3) * 32) >> 4);
+                                tc::mma_bf16_ss(d, qd + off, kd + off, idesc_s, k > 0);
+                            }
+                            tc::mma_commit(&s_full[j]);
+                            if (j == 1) {
+                                tc::mma_commit(&k_empty[ks]);
+                                if (tn == it.ntiles - 1) tc::mma_commit(q_empty);
+                            }
                         }
-                        tc::mma_commit(&s_full[T & 1]);
-                        tc::mma_commit(&k_empty[ks]);
-                        if (ts == it.ntiles - 1) tc::mma_commit(q_empty);
+                        __syncwarp();
                     }
-                    __syncwarp();
                 }
             }
             kv_iter += it.ntiles;
@@ -562,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else if (warp >= kFirstSoftmaxWarp) {
-        // ==== softmax: warpgroup j (warps 4 + 4 j .. 7 + 4 j) takes the KV tiles T with T % 2 == j ====
+        // ==== softmax: warpgroup j (warps 4 + 4 j .. 7 + 4 j) owns Q tile j of every item ====
         // Registers: the launch gives every thread 168; the first warpgroup (MMA,
         // producers) drops to 56 so that a softmax thread can hold a whole
         // 128-key S row: 128 x 56 + 256 x 224 = 384 x 168.
@@ -570,8 +583,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int j = (warp - kFirstSoftmaxWarp) >> 2;
         const int row = (warp & 3) * 32 + lane;  // warp % 4 selects the TMEM lane quarter
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t s_cols = tmem + lane_off + j * kTileN;  // S_j, then P_j over its first 64 columns
-        const uint32_t o_cols = tmem + lane_off + kTmemO;      // O_0 at +0, O_1 at +D
+        const uint32_t s_cols = tmem + lane_off + j * kTileN;   // S_j, then P_j over its first 64 columns
+        const uint32_t o_cols = tmem + lane_off + kTmemO + j * 128;
         const float sl2 = p.scale_log2;
         uint32_t kv_iter = 0, item_iter = 0;
         for (long long r = 0; r < rounds; ++r) {
@@ -579,15 +592,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (idx >= n_items) break;
             const Item it = load_item<G>(p, idx);
             const int pos = row / G, jh = row % G;
-            const bool valid_row = pos < it.npos;
-            const int lim_min = it.L - it.n + it.p0;  // smallest limit among the tile's rows
-            // rows past the tile's positions attend like its first row (their output is dropped)
-            const int lim = valid_row ? (lim_min + pos) : lim_min;
-            const int t_first = (int)((j - (int)(kv_iter & 1)) & 1);  // first tile of this warpgroup
+            const int p0 = it.p0 + j * ppt;  // first position of this Q tile
+            const int npos = j == 0 ? it.npos_a : it.npos_b;
+            const bool valid_row = pos < npos;
+            // rows past the tile's positions attend like its first row (their output is
+            // dropped); no row's keys reach past the item's last key
+            const int lim_min = min(it.L - it.n + p0, it.kv_end - 1);
+            const int lim = min(valid_row ? (it.L - it.n + p0 + pos) : lim_min, it.kv_end - 1);
             float m = -INFINITY, l = 0.f;
-            for (int t = t_first; t < it.ntiles; t += 2) {
+            for (int t = 0; t < it.ntiles; ++t) {
                 const uint32_t T = kv_iter + t;
-                NPV_WAIT(&s_full[j], (T >> 1) & 1);
+                NPV_WAIT(&s_full[j], T & 1);
                 tc::fence_after_sync();
                 float sv[kTileN];
                 {
@@ -620,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // 2^kRescaleThreshold; O_j is then rescaled after P is written
                 float alpha = 1.0f;
                 bool rescale = false;
-                if (t == t_first) {
+                if (t == 0) {
                     m = m_tile;
                 } else {
                     const float m_new = fmaxf(m, m_tile);
@@ -649,12 +664,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
                 if (rescale) {
-                    // O_j: its last P.V finished before S_t (issued after it) completed,
-                    // and the next one waits for p_full below
+                    // O_j: its last P.V (PV_j(t-1)) finished before S_j(t), issued after
+                    // it, completed; the next one waits for p_full below
 #pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t raw[32];
-                        const uint32_t ta = o_cols + j * D + c * 32;
+                        const uint32_t ta = o_cols + c * 32;
                         tc::tmem_ld32(ta, raw);
                         tc::tmem_wait_ld();
 #pragma unroll
@@ -667,46 +682,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&p_full[j]);
             }
-            // ---- epilogue: merge the two warpgroups' partial results, O / l -> bf16
-            // (double-buffered by item parity: the other warpgroup may still read
-            // this item's slot when this one reaches the next item's epilogue; the
-            // mbarrier's release / acquire orders these global accesses in the CTA)
-            float2 *xml_item = xml + (item_iter & 1) * 2 * kTileM;
-            xml_item[j * kTileM + row] = make_float2(m, l);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(ml_full);
-            NPV_WAIT(ml_full, item_iter & 1);
-            NPV_WAIT(o_full, item_iter & 1);
+            // ---- epilogue: O_j / l -> bf16 rows of this Q tile
+            NPV_WAIT(&o_full[j], item_iter & 1);
             tc::fence_after_sync();
             {
-                const float2 mo = xml_item[(1 - j) * kTileM + row];
-                const bool has_me = t_first < it.ntiles, has_other = (1 - t_first) < it.ntiles;
-                float mm = fmaxf(has_me ? m : -INFINITY, has_other ? mo.x : -INFINITY);
-                const float a_me = has_me ? fast_exp2(m - mm) : 0.f;
-                const float a_ot = has_other ? fast_exp2(mo.x - mm) : 0.f;
-                const float inv = 1.0f / (a_me * l + a_ot * mo.y);
-                const float a0 = j == 0 ? a_me : a_ot, a1 = j == 0 ? a_ot : a_me;
-                const bool has0 = j == 0 ? has_me : has_other, has1 = j == 0 ? has_other : has_me;
-                // this warpgroup writes output columns [j D / 2, (j + 1) D / 2)
-                uint16_t *orow = p.out + ((int64_t)(it.row0 + it.p0 + pos) * p.num_q_heads + it.h * G + jh) * D +
-                                 j * (D / 2);
+                const float inv = 1.0f / l;
+                uint16_t *orow = p.out + ((int64_t)(it.row0 + p0 + pos) * p.num_q_heads + it.h * G + jh) * D;
 #pragma unroll
-                for (int c = 0; c < D / 64; ++c) {
-                    uint32_t r0[32], r1[32];
-                    const uint32_t col = j * (D / 2) + c * 32;
-                    if (has0) tc::tmem_ld32(o_cols + col, r0);
-                    if (has1) tc::tmem_ld32(o_cols + D + col, r1);
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r32[32];
+                    tc::tmem_ld32(o_cols + c * 32, r32);
                     tc::tmem_wait_ld();
                     if (valid_row) {
 #pragma unroll
                         for (int v = 0; v < 4; ++v) {
                             float f[8];
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                const float x0 = has0 ? __uint_as_float(r0[v * 8 + e]) * a0 : 0.f;
-                                const float x1 = has1 ? __uint_as_float(r1[v * 8 + e]) * a1 : 0.f;
-                                f[e] = (x0 + x1) * inv;
-                            }
+                            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r32[v * 8 + e]) * inv;
                             st_global_v4(orow + c * 32 + v * 8, pack8(f));
                         }
                     }
