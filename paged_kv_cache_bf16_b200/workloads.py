@@ -439,10 +439,11 @@ PROFILE_SPECS: Dict[str, Spec] = {
         block_size=256, num_blocks=1024, ctx_lo=100, ctx_hi=2048, num_steps=4,
         description="qwen3_decode with 64 sequences and a 1,024-block pool (profiling size)"),
     "chunked_prefill_small": Spec(
-        name="chunked_prefill_small", seed=5, num_seqs=68, num_q_heads=16, num_kv_heads=8, head_dim=128,
-        block_size=256, num_blocks=1024, ctx_lo=100, ctx_hi=2048, prefill_seqs=4, prefill_len=512,
+        name="chunked_prefill_small", seed=5, num_seqs=32, num_q_heads=16, num_kv_heads=8, head_dim=128,
+        block_size=256, num_blocks=1024, ctx_lo=100, ctx_hi=2048, prefill_seqs=16, prefill_len=512,
         prior_lo=0, prior_hi=8192,
-        description="chunked_prefill_mixed with 4 prefill + 64 decode sequences (profiling size)"),
+        description="chunked_prefill_mixed with all 16 prefill sequences but 16 decode sequences and a "
+                    "1,024-block pool (profiling size: 1 GB of cache on the device)"),
 }
 
 
