@@ -79,7 +79,9 @@ typedef enum {
 #define NPV_DEVERR_BLOCK_ID 0x2u    /* a live block-table entry outside [0, num_blocks) */
 #define NPV_DEVERR_CONTEXT_LEN 0x4u /* context length < 0, > max_blocks_per_seq * block_size,
                                        or smaller than the sequence's query rows */
-#define NPV_DEVERR_QUERY_LENS 0x8u  /* cu_seqlens_q not nondecreasing from 0 to total_q */
+#define NPV_DEVERR_QUERY_LENS 0x8u  /* cu_seqlens_q not nondecreasing from 0 to total_q, or an
+                                       n_b above a max_seqlen_q that sent the call to the
+                                       decode kernel alone */
 #define NPV_DEVERR_TIMEOUT 0x10u    /* an internal pipeline wait gave up after ~2 s (library bug) */
 
 /* Static description of a status code. Never NULL. */
@@ -204,11 +206,15 @@ NPV_API size_t npv_paged_prefill_workspace_size(int32_t num_seqs, int32_t total_
  *                 including its n_b new rows, which must already be stored.
  *                 Row i of sequence b sits at position L_b - n_b + i and sees
  *                 keys 0 .. L_b - n_b + i.  L_b < n_b sets NPV_DEVERR_CONTEXT_LEN.
- *   max_seqlen_q  host upper bound on n_b, the flash-attn-style hint; checked to be
- *                 >= 0.  When max_seqlen_q * g <= 8 the short sequences run on a
- *                 lighter variant of the decode kernel (see below); the row
- *                 counts themselves are read on the device, so a wrong hint
- *                 changes only which kernel serves a sequence, not the result.
+ *   max_seqlen_q  host upper bound on every n_b, as in flash-attn's varlen calls;
+ *                 checked to be >= 0.  When max_seqlen_q * g <= 8 the short
+ *                 sequences run on a lighter variant of the decode kernel (see
+ *                 below).  When max_seqlen_q <= m every sequence fits the decode
+ *                 kernel, and the call launches that kernel alone (no tcgen05
+ *                 kernel, no plan); a sequence with n_b > m then sets
+ *                 NPV_DEVERR_QUERY_LENS and its rows are written as zeros.  With
+ *                 max_seqlen_q > m a bound that is broken costs nothing: the row
+ *                 counts are read on the device and route each sequence.
  *   other arguments as for npv_paged_decode_attention.
  * Sequences with n_b > m (g = num_q_heads / num_kv_heads; m = 8 / g when
  * max_seqlen_q * g <= 8, else 16 / g) run on the tcgen05 tensor cores (QK^T and

@@ -81,6 +81,8 @@ struct Params {
     int32_t total_q;              // rows of q and out in a mixed batch
     int32_t max_rows;             // most query rows of a sequence on this path (1 without cu_seqlens_q)
     int32_t rows_per_head;        // RP: query-row slots per KV head in a partial slot (g * max_rows)
+    int32_t sole_path;            // mixed batch served by this kernel alone: a sequence of more than
+                                  // max_rows rows, or a malformed range, is reported here
     int32_t max_blocks_per_seq;
     int32_t num_seqs;
     int32_t num_q_heads;
@@ -126,6 +128,23 @@ __device__ __forceinline__ int32_t seq_chunks(const Params &p, int32_t b) {
 
 __device__ __forceinline__ int64_t query_row(const Params &p, int32_t b) {
     return p.cu_seqlens_q != nullptr ? (int64_t)__ldg(p.cu_seqlens_q + b) : (int64_t)b;
+}
+
+// In a mixed batch that this kernel serves alone (the caller's bound on the
+// query rows fits its tile), sequence b with no rows on this path is either
+// empty, malformed (NPV_DEVERR_QUERY_LENS) or longer than the bound: its rows
+// are written as zeros and NPV_DEVERR_QUERY_LENS is reported.
+__device__ __forceinline__ void reject_foreign_rows(const Params &p, int32_t b, int head_dim) {
+    const int32_t cb = __ldg(p.cu_seqlens_q + b), ce = __ldg(p.cu_seqlens_q + b + 1);
+    if (cb < 0 || ce < cb || ce > p.total_q) {
+        report_error(NPV_DEVERR_QUERY_LENS);
+        return;
+    }
+    if (ce - cb <= p.max_rows) return;  // empty
+    report_error(NPV_DEVERR_QUERY_LENS);
+    uint4 *o = reinterpret_cast<uint4 *>(p.out + (int64_t)cb * p.num_q_heads * head_dim);
+    const int64_t nvec = (int64_t)(ce - cb) * p.num_q_heads * head_dim / 8;
+    for (int64_t i = 0; i < nvec; ++i) o[i] = make_uint4(0, 0, 0, 0);
 }
 
 // Exclusive prefix sum over the block; returns the exclusive value and sets *total.
@@ -698,12 +717,21 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const Params p, int h
 
     const Schedule sc = compute_schedule(p, sched, scratch);
 
+    // (0) with no prefill kernel in the call, its check that cu_seqlens_q runs
+    // from 0 to total_q is made here
+    if (p.sole_path && c == 0 && threadIdx.x == 0 &&
+        (__ldg(p.cu_seqlens_q) != 0 || __ldg(p.cu_seqlens_q + p.num_seqs) != p.total_q))
+        report_error(NPV_DEVERR_QUERY_LENS);
+
     // (1) rows of this path's sequences with no chunks
     for (long long b = c + G * threadIdx.x; b < p.num_seqs; b += G * blockDim.x) {
         const int32_t n = path_rows(p, (int32_t)b);
-        // other sequences belong to the prefill kernel, which also reports
-        // malformed cu_seqlens_q
-        if (n == 0) continue;
+        if (n == 0) {
+            // other sequences belong to the prefill kernel, which also reports
+            // malformed cu_seqlens_q, unless this call runs no prefill kernel
+            if (p.sole_path) reject_foreign_rows(p, (int32_t)b, D);
+            continue;
+        }
         const int32_t L = __ldg(p.context_lens + b);
         const bool bad = L < 0 || (long long)L > (long long)p.max_blocks_per_seq * p.block_size ||
                          (p.cu_seqlens_q != nullptr && L < n);

@@ -78,6 +78,7 @@ struct DecodeConfig {
     int head_groups = 0;     // Hkv / HC
     int max_rows = 0;        // most query rows of a sequence the kernel serves
     int rows_per_head = 0;   // partial-slot rows per KV head: g * max_rows
+    bool sole_path = false;  // mixed batch with no prefill kernel launched
     int stages = 0;
     int grid = 0;
     size_t smem = 0;
@@ -194,6 +195,7 @@ npv_status run_decode(void *out, const void *q, int64_t q_row_stride, const int3
     p.num_head_groups = cfg.head_groups;
     p.max_rows = cfg.max_rows;
     p.rows_per_head = cfg.rows_per_head;
+    p.sole_path = cfg.sole_path ? 1 : 0;
     p.num_stages = cfg.stages;
     const float s = scale > 0.f ? scale : (float)(1.0 / std::sqrt((double)head_dim));
     p.scale_log2 = s * 1.4426950408889634f;
@@ -476,49 +478,52 @@ npv_status npv_paged_prefill_attention(void *out, const void *q, const int32_t *
     cudaStream_t s = (cudaStream_t)stream;
     const int D = head_dim, G = cfg.decode.group;
 
-    // tensor maps, 128-byte swizzle: the caches [NB * BS, Hkv, D] in boxes of
-    // {64 elements, 1 head, box_tokens slots}; q [total_q, Hq, D] in boxes of
-    // {64 elements, G heads, 128 / G positions} (one 128-row tile of a KV head)
-    CUtensorMap qmap, kmap, vmap;
-    const int box_tokens = (block_size % 128 == 0) ? 128 : 16;
-    if (!encode_map_3d(&qmap, q, D, num_q_heads, (uint64_t)total_q, 64, G, npv::prefill::kTileM / G) ||
-        !encode_map_3d(&kmap, k_cache, D, num_kv_heads, (uint64_t)num_blocks * block_size, 64, 1, box_tokens) ||
-        !encode_map_3d(&vmap, v_cache, D, num_kv_heads, (uint64_t)num_blocks * block_size, 64, 1, box_tokens))
-        return NPV_ERR_CUDA;
-
-    npv::prefill::Params p = {};
-    p.out = static_cast<uint16_t *>(out);
-    p.cu_seqlens_q = cu_seqlens_q;
-    p.context_lens = context_lens;
-    p.block_tables = block_tables;
-    p.total_q = total_q;
-    p.num_seqs = num_seqs;
-    p.num_q_heads = num_q_heads;
-    p.num_kv_heads = num_kv_heads;
-    p.num_blocks = num_blocks;
-    p.block_size = block_size;
-    p.max_blocks_per_seq = max_blocks_per_seq;
-    p.box_tokens = box_tokens;
-    p.q = static_cast<const uint16_t *>(q);
-    const float sc = scale > 0.f ? scale : (float)(1.0 / std::sqrt((double)head_dim));
-    p.scale_log2 = sc * 1.4426950408889634f;
-    char *ws = static_cast<char *>(workspace);
-    p.plan_count = reinterpret_cast<int32_t *>(ws + cfg.decode.ws_total);
-    p.plan_pairs = reinterpret_cast<int2 *>(ws + cfg.decode.ws_total + 256);
-    p.max_pairs = cfg.max_pairs;
-
     // The decode kernel takes the sequences whose g * n_b rows fit its MMA
     // columns: one 8-column tile when max_seqlen_q says that suffices (fewer
-    // registers), else two.  The hint only moves sequences between the two
-    // kernels, which both routes use alike, so a wrong hint costs speed, never
-    // correctness.
+    // registers), else two.  The row counts themselves are read on the device.
     if ((int64_t)max_seqlen_q * G <= 8) {
         cfg.decode.max_rows = 8 / G;
         cfg.decode.rows_per_head = 8;
     }
-    p.decode_rows_max = cfg.decode.max_rows;
-    cudaError_t e = dispatch_prefill(D, G, p, qmap, kmap, vmap, cfg, s);
-    if (e != cudaSuccess) return NPV_ERR_CUDA;
+    // When the hint bounds every sequence by the decode kernel's rows, no
+    // sequence is left for the tensor-memory kernel: its plan and launch are
+    // skipped, and the decode kernel reports a sequence that breaks the bound.
+    cfg.decode.sole_path = max_seqlen_q <= cfg.decode.max_rows;
+    if (!cfg.decode.sole_path) {
+        // tensor maps, 128-byte swizzle: the caches [NB * BS, Hkv, D] in boxes of
+        // {64 elements, 1 head, box_tokens slots}; q [total_q, Hq, D] in boxes of
+        // {64 elements, G heads, 128 / G positions} (one 128-row tile of a KV head)
+        CUtensorMap qmap, kmap, vmap;
+        const int box_tokens = (block_size % 128 == 0) ? 128 : 16;
+        if (!encode_map_3d(&qmap, q, D, num_q_heads, (uint64_t)total_q, 64, G, npv::prefill::kTileM / G) ||
+            !encode_map_3d(&kmap, k_cache, D, num_kv_heads, (uint64_t)num_blocks * block_size, 64, 1, box_tokens) ||
+            !encode_map_3d(&vmap, v_cache, D, num_kv_heads, (uint64_t)num_blocks * block_size, 64, 1, box_tokens))
+            return NPV_ERR_CUDA;
+
+        npv::prefill::Params p = {};
+        p.out = static_cast<uint16_t *>(out);
+        p.cu_seqlens_q = cu_seqlens_q;
+        p.context_lens = context_lens;
+        p.block_tables = block_tables;
+        p.total_q = total_q;
+        p.num_seqs = num_seqs;
+        p.num_q_heads = num_q_heads;
+        p.num_kv_heads = num_kv_heads;
+        p.num_blocks = num_blocks;
+        p.block_size = block_size;
+        p.max_blocks_per_seq = max_blocks_per_seq;
+        p.box_tokens = box_tokens;
+        p.q = static_cast<const uint16_t *>(q);
+        const float sc = scale > 0.f ? scale : (float)(1.0 / std::sqrt((double)head_dim));
+        p.scale_log2 = sc * 1.4426950408889634f;
+        char *ws = static_cast<char *>(workspace);
+        p.plan_count = reinterpret_cast<int32_t *>(ws + cfg.decode.ws_total);
+        p.plan_pairs = reinterpret_cast<int2 *>(ws + cfg.decode.ws_total + 256);
+        p.max_pairs = cfg.max_pairs;
+        p.decode_rows_max = cfg.decode.max_rows;
+        cudaError_t e = dispatch_prefill(D, G, p, qmap, kmap, vmap, cfg, s);
+        if (e != cudaSuccess) return NPV_ERR_CUDA;
+    }
     // sequences of 1 .. 16 / g query rows: the split-KV decode kernel
     return run_decode(out, q, (int64_t)num_q_heads * head_dim, cu_seqlens_q, total_q, k_cache, v_cache,
                       block_tables, max_blocks_per_seq, context_lens, num_seqs, num_q_heads, num_kv_heads,

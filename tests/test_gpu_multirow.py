@@ -3,7 +3,8 @@ prefill call, against the fp64 oracle (GPU).
 
 Sequences with g * n_b <= 16 query rows per KV head run on the split-KV decode
 kernel's warp-level MMA tiles (one 8-column tile when the call's max_seqlen_q
-hint says g * n_b <= 8, two otherwise); longer ones on the tcgen05 kernel.  Each
+bound says g * n_b <= 8, two otherwise); longer ones on the tcgen05 kernel.  A
+bound that fits the decode tile runs that kernel alone.  Each
 call here mixes decode rows, short multi-row sequences and longer chunks, with
 contexts long enough that most (sequence, KV head) units are cut across CTAs
 and merged.  Every row is checked; a row i of a sequence with n_b rows and
@@ -49,22 +50,57 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("hint", ["max", "one"])
 @pytest.mark.parametrize("case", CASES, ids=lambda c: "D%d_q%d_kv%d_bs%d" % c)
-def test_mixed_row_counts_in_one_call(case, hint):
+def test_mixed_row_counts_in_one_call(case):
     D, Hq, Hkv, BS = case
     wl = _workload(4000 + sum(case), D, Hq, Hkv, BS, QLENS)
     st = W.DeviceState(wl, DEV)
     run_store(st, 0)
     s = st.steps[0]
-    # the hint picks the one- or two-tile decode variant; "one" under-states it,
-    # which sends the longer short sequences to the tcgen05 kernel instead
-    mq = int(wl.query_lens.max()) if hint == "max" else 1
+    mq = int(wl.query_lens.max())
     out = ops.paged_prefill_attention(s["q"], st.k_cache, st.v_cache, s["cu_seqlens_q"], mq, s["block_tables"],
                                       s["context_lens"])
     no_device_errors()
     ref, rows = oracle_compact(wl, 0)
-    assert_close(out[torch.from_numpy(rows).to(DEV)], ref, f"{case} hint={hint}")
+    assert_close(out[torch.from_numpy(rows).to(DEV)], ref, f"{case}")
+
+
+def _decode_rows_limit(g, max_seqlen_q):
+    """Most query rows per sequence the decode kernel takes (its MMA columns)."""
+    return 8 // g if max_seqlen_q * g <= 8 else 16 // g
+
+
+@pytest.mark.parametrize("mq", [1, 2, 4])
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "D%d_q%d_kv%d_bs%d" % c)
+def test_bound_within_decode_tile(case, mq):
+    """max_seqlen_q <= m: the call runs the decode kernel alone.  Sequences within
+    its m rows are exact; a longer one (the bound broken) reports
+    NPV_DEVERR_QUERY_LENS and its rows are zeros."""
+    D, Hq, Hkv, BS = case
+    g = Hq // Hkv
+    m = _decode_rows_limit(g, mq)
+    if mq > m:
+        pytest.skip("this bound sends long sequences to the tcgen05 kernel")
+    wl = _workload(4200 + sum(case) + mq, D, Hq, Hkv, BS, QLENS)
+    st = W.DeviceState(wl, DEV)
+    run_store(st, 0)
+    s = st.steps[0]
+    out = ops.paged_prefill_attention(s["q"], st.k_cache, st.v_cache, s["cu_seqlens_q"], mq, s["block_tables"],
+                                      s["context_lens"])
+    long_seq = wl.query_lens > m
+    assert long_seq.any()
+    with pytest.raises(ops.NpvError) as ei:
+        ops.check_device_errors()
+    assert ei.value.bits == 0x8, ei.value.bits
+    ref, rows = oracle_compact(wl, 0)
+    cu = wl.cu_seqlens_q()
+    owner = np.searchsorted(cu, rows, side="right") - 1
+    keep = ~long_seq[owner]
+    got = out[torch.from_numpy(rows).to(DEV)]
+    assert_close(got[torch.from_numpy(keep).to(DEV)], ref[keep], f"{case} mq={mq} in-bound rows")
+    dropped = got[torch.from_numpy(~keep).to(DEV)]
+    assert dropped.numel() > 0 and torch.count_nonzero(dropped).item() == 0
+    no_device_errors()
 
 
 @pytest.mark.parametrize("n", [2, 4, 8])
@@ -91,3 +127,24 @@ def test_verify_rows_equal_single_row_problems(n):
     assert np.array_equal(rows, np.arange(int(cu[-1])))
     assert_close(out, ref, "verify rows")
     assert_close(dec, ref, "as decode rows")
+
+
+def test_malformed_query_ranges_on_decode_only_call():
+    """With the decode kernel alone in the call, a cu_seqlens_q with a decreasing
+    entry or a first entry other than 0 still sets NPV_DEVERR_QUERY_LENS, and the
+    next call is exact."""
+    wl = _workload(4300, 128, 16, 8, 256, [2, 1, 1, 4], hi=600)
+    st = W.DeviceState(wl, DEV)
+    run_store(st, 0)
+    s = st.steps[0]
+    for cu in ([0, 3, 2, 4, 8], [1, 2, 3, 4, 8], [0, 2, 3, 4, 7]):
+        bad = torch.tensor(cu, dtype=torch.int32, device=DEV)
+        ops.paged_prefill_attention(s["q"], st.k_cache, st.v_cache, bad, 4, s["block_tables"], s["context_lens"])
+        with pytest.raises(ops.NpvError) as ei:
+            ops.check_device_errors()
+        assert ei.value.bits & 0x8, cu
+    out = ops.paged_prefill_attention(s["q"], st.k_cache, st.v_cache, s["cu_seqlens_q"], 4, s["block_tables"],
+                                      s["context_lens"])
+    no_device_errors()
+    ref, rows = oracle_compact(wl, 0)
+    assert_close(out[torch.from_numpy(rows).to(DEV)], ref, "after malformed decode-only calls")
