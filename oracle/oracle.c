@@ -30,6 +30,13 @@
  *            The FlashAttention family (README, Features) only re-arranges this
  *            result, so the oracle is the plain definition.
  *
+ *   rope     "Nano-vLLM Architecture and Performance", project structure
+ *            (layers/rotary_embedding.py: RoPE, the rotary position embedding
+ *            applied to q and k before the attention layer stores k).  The
+ *            pages name the step only; oracle_rope states the rotary embedding
+ *            of Su et al., "RoFormer" (2021), section 3.4, in the rotate-half
+ *            pairing of dimension i with i + D/2 that Qwen3 uses.
+ *
  * Readings where the pages are silent (each also listed in the design notes):
  *   - slot s addresses block s / block_size, offset s % block_size;
  *   - a negative slot is a padding row and writes nothing;
@@ -298,4 +305,72 @@ int oracle_paged_attention(double *out, const uint16_t *q, const int32_t *cu_seq
             pthread_join(tid[t], NULL);
     }
     return job.error;
+}
+
+/*
+ * Rotary position embedding of num_tokens x num_heads rows of head_dim bf16
+ * values (token rows token_stride elements apart), written to out as fp64
+ * [num_tokens][num_heads][head_dim].  Token t sits at position p = positions[t];
+ * for i < D/2 the pair (x[i], x[i + D/2]) is turned by the angle p * theta_i,
+ * theta_i = base^(-2i/D):
+ *     out[i]       = x[i] cos(p theta_i) - x[i + D/2] sin(p theta_i)
+ *     out[i + D/2] = x[i + D/2] cos(p theta_i) + x[i] sin(p theta_i)
+ * i.e. the complex number x[i] + j x[i + D/2] times exp(j p theta_i).
+ */
+int oracle_rope(double *out, const uint16_t *x, int64_t num_tokens, int32_t num_heads, int32_t head_dim,
+                int64_t token_stride, const int32_t *positions, double base)
+{
+    if (num_tokens < 0 || num_heads <= 0 || head_dim <= 0 || head_dim % 2 != 0 || !(base > 0.0))
+        return ORACLE_ERR_ARG;
+    if (token_stride < (int64_t)num_heads * head_dim)
+        return ORACLE_ERR_ARG;
+    if (num_tokens == 0)
+        return ORACLE_OK;
+    if (!out || !x || !positions)
+        return ORACLE_ERR_ARG;
+    const int32_t half = head_dim / 2;
+    for (int64_t t = 0; t < num_tokens; ++t) {
+        const double p = (double)positions[t];
+        for (int32_t i = 0; i < half; ++i) {
+            const double theta = pow(base, -2.0 * (double)i / (double)head_dim);
+            const double angle = p * theta;
+            const double c = cos(angle), s = sin(angle);
+            for (int32_t h = 0; h < num_heads; ++h) {
+                const uint16_t *row = x + t * token_stride + (int64_t)h * head_dim;
+                double *o = out + (t * num_heads + h) * (int64_t)head_dim;
+                const double x1 = bf16_to_double(row[i]);
+                const double x2 = bf16_to_double(row[i + half]);
+                o[i] = x1 * c - x2 * s;
+                o[i + half] = x2 * c + x1 * s;
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * The bf16 value nearest to v, ties to even (IEEE 754 round-to-nearest for an
+ * 8-bit significand with fp32's exponent range); NaN gives the quiet NaN 0x7FC0
+ * and magnitudes that round past the largest finite value give infinity.
+ */
+uint16_t oracle_double_to_bf16(double v)
+{
+    if (isnan(v))
+        return 0x7FC0;
+    const uint16_t sign = signbit(v) ? 0x8000 : 0;
+    const double a = fabs(v);
+    if (a == 0.0)
+        return sign;
+    int e;
+    frexp(a, &e);          /* a = m 2^e with 0.5 <= m < 1 */
+    int q = e - 8;         /* spacing of the 8-bit significands in [2^(e-1), 2^e) */
+    if (q < -133)
+        q = -133;          /* subnormal spacing, 2^-126 / 2^7 */
+    const double y = ldexp(nearbyint(ldexp(a, -q)), q);
+    if (y > ldexp(255.0, 120))  /* largest finite bf16: (2 - 2^-7) 2^127 */
+        return sign | 0x7F80;
+    const float f = (float)y;   /* exact: at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(sign | (u >> 16));
 }

@@ -49,6 +49,10 @@ def load(path: str) -> C.CDLL:
     l.oracle_paged_attention.restype = C.c_int
     l.oracle_bf16_to_double.argtypes = [C.c_uint16]
     l.oracle_bf16_to_double.restype = C.c_double
+    l.oracle_rope.argtypes = [p, p, C.c_int64, i32, i32, C.c_int64, p, C.c_double]
+    l.oracle_rope.restype = C.c_int
+    l.oracle_double_to_bf16.argtypes = [C.c_double]
+    l.oracle_double_to_bf16.restype = C.c_uint16
     return l
 
 
@@ -123,3 +127,38 @@ def decode_attention(q: np.ndarray, k_pool: np.ndarray, v_pool: np.ndarray, bloc
 def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
     """Widen bf16 bit patterns to float64 (exact)."""
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def rope(x: np.ndarray, positions: np.ndarray, base: float, _lib: Optional[C.CDLL] = None) -> np.ndarray:
+    """fp64 rotary embedding of bf16 rows x [T, H, D] at positions [T] (rotate-half pairing)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    pos = np.ascontiguousarray(positions, dtype=np.int32)
+    T, H, D = x.shape
+    assert pos.shape == (T,)
+    out = np.zeros((T, H, D), dtype=np.float64)
+    _check((_lib or lib()).oracle_rope(_ptr(out), _ptr(x), T, H, D, H * D, _ptr(pos), float(base)))
+    return out
+
+
+def to_bf16(v: np.ndarray, _lib: Optional[C.CDLL] = None) -> np.ndarray:
+    """Round fp64 values to bf16 bit patterns, nearest with ties to even."""
+    f = (_lib or lib()).oracle_double_to_bf16
+    flat = np.asarray(v, dtype=np.float64).ravel()
+    return np.fromiter((f(float(a)) for a in flat), dtype=np.uint16, count=flat.size).reshape(np.shape(v))
+
+
+def rope_store_kvcache(q: Optional[np.ndarray], key: np.ndarray, value: np.ndarray, positions: np.ndarray,
+                       k_pool: np.ndarray, v_pool: np.ndarray, slot_mapping: np.ndarray, base: float,
+                       _lib: Optional[C.CDLL] = None):
+    """RoPE on q and key, then the store of the rotated key and the value.
+
+    The tensors are bf16, so the rotated rows are the bf16 roundings of the fp64
+    rotations.  Returns (q rotated [T, Hq, D] bf16 bits or None, fp64 rotated q,
+    fp64 rotated key); the pools are updated in place.
+    """
+    kr = rope(key, positions, base, _lib)
+    store_kvcache(to_bf16(kr, _lib), value, k_pool, v_pool, slot_mapping, _lib=_lib)
+    if q is None:
+        return None, None, kr
+    qr = rope(q, positions, base, _lib)
+    return to_bf16(qr, _lib), qr, kr

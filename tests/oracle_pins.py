@@ -17,11 +17,16 @@ catch.  What pins what:
   chunking       one chunk equals two successive chunks; a prefill row equals
                  decode over the truncated context
   prefix sharing shared physical blocks equal private copies
+  rope           unit vectors at whole-radian angles (tests/golden/rope_worked_example.txt);
+                 the complex-product form with numpy's complex exponential; the
+                 relative-position identity and pair lengths; position 0 is the identity
+  bf16 rounding  the input generator's fp32 bit-level rounding; hand-worked ties and limits
 """
 
 from __future__ import annotations
 
 import math
+import os
 
 import numpy as np
 
@@ -335,10 +340,115 @@ def check_threads_agree(lib) -> None:
     assert np.array_equal(a, b)
 
 
+# ------------------------------------------------------------------ rope ----
+
+ROPE_GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "rope_worked_example.txt")
+
+
+def rope_golden_rows():
+    rows = []
+    for line in open(ROPE_GOLDEN):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        f = line.split()
+        D, base, pos, unit = int(f[0]), float(f[1]), int(f[2]), int(f[3])
+        expect = np.array([float(v) for v in f[4:]])
+        assert expect.shape == (D,)
+        rows.append((D, base, pos, unit, expect))
+    return rows
+
+
+def check_rope_worked_example(lib) -> None:
+    """Unit vectors at positions where p * theta_i is a whole number of radians."""
+    rows = rope_golden_rows()
+    assert len(rows) >= 10
+    for D, base, pos, unit, expect in rows:
+        x = np.zeros((1, 1, D), dtype=np.float32)
+        x[0, 0, unit] = 1.0
+        out = O.rope(_bits(x), np.array([pos], dtype=np.int32), base, _lib=lib)[0, 0]
+        assert np.max(np.abs(out - expect)) < 1e-14, (D, base, pos, unit, out, expect)
+
+
+def check_rope_position_zero(lib) -> None:
+    rng = np.random.default_rng(31)
+    x = _bits(rng.standard_normal((4, 3, 64)))
+    out = O.rope(x, np.zeros(4, dtype=np.int32), 1.0e6, _lib=lib)
+    assert np.array_equal(out, _f64(x))
+
+
+def check_rope_complex_product(lib) -> None:
+    """The rotation is the complex product z_i exp(j p theta_i), z_i = x_i + j x_{i+D/2}
+    (numpy's complex exponential; theta_i = base^(-2i/D), RoFormer section 3.4)."""
+    rng = np.random.default_rng(32)
+    pos = np.array([0, 1, 7, 4095, 40959, 131071], dtype=np.int32)
+    for D in (8, 64, 128):
+        for base in (1.0e4, 1.0e6):
+            x = _bits(rng.standard_normal((pos.size, 3, D)))
+            f = _f64(x)
+            h = D // 2
+            theta = np.power(base, -np.arange(h, dtype=np.float64) * 2.0 / D)
+            w = (f[..., :h] + 1j * f[..., h:]) * np.exp(1j * pos[:, None, None].astype(np.float64) * theta)
+            expect = np.concatenate([w.real, w.imag], axis=-1)
+            out = O.rope(x, pos, base, _lib=lib)
+            assert np.max(np.abs(out - expect)) < 1e-9, (D, base, np.max(np.abs(out - expect)))
+
+
+def check_rope_relative_position(lib) -> None:
+    """<R(m) q, R(n) k> = <R(m - n) q, k> (the property RoPE is built for) and each
+    pair keeps its length."""
+    rng = np.random.default_rng(33)
+    D = 64
+    q = _bits(rng.standard_normal((1, 4, D)))
+    k = _bits(rng.standard_normal((1, 4, D)))
+    for m, n in ((5, 3), (1000, 17), (70000, 69999), (12, 40)):
+        qm = O.rope(q, np.array([m], dtype=np.int32), 1.0e6, _lib=lib)
+        kn = O.rope(k, np.array([n], dtype=np.int32), 1.0e6, _lib=lib)
+        qd = O.rope(q, np.array([m - n], dtype=np.int32), 1.0e6, _lib=lib)
+        lhs = np.sum(qm * kn, axis=-1)
+        rhs = np.sum(qd * _f64(k), axis=-1)
+        assert np.max(np.abs(lhs - rhs)) < 1e-9, (m, n, lhs, rhs)
+        h = D // 2
+        r_in = _f64(q)[..., :h] ** 2 + _f64(q)[..., h:] ** 2
+        r_out = qm[..., :h] ** 2 + qm[..., h:] ** 2
+        assert np.max(np.abs(r_in - r_out)) < 1e-12
+
+
+def check_rope_strided_rows(lib) -> None:
+    """Rows are read token_stride apart and heads D apart: a token's heads and tokens
+    do not mix (each [head] slice equals a one-head call on that slice)."""
+    rng = np.random.default_rng(34)
+    x = _bits(rng.standard_normal((5, 3, 16)))
+    pos = np.array([3, 0, 9, 2, 7], dtype=np.int32)
+    out = O.rope(x, pos, 1.0e4, _lib=lib)
+    for t in range(5):
+        for h in range(3):
+            one = O.rope(x[t:t + 1, h:h + 1], pos[t:t + 1], 1.0e4, _lib=lib)[0, 0]
+            assert np.array_equal(out[t, h], one), (t, h)
+
+
+def check_to_bf16(lib) -> None:
+    """Nearest bf16, ties to even: agrees with the bit-level fp32 rounding of the input
+    generator on fp32-exact values, and on hand-worked ties and limits."""
+    rng = np.random.default_rng(35)
+    v = (rng.standard_normal(4096) * np.exp2(rng.integers(-140, 120, 4096))).astype(np.float32)
+    assert np.array_equal(O.to_bf16(v.astype(np.float64), _lib=lib), W.f32_to_bf16_bits(v))
+    cases = {
+        1.0: 0x3F80, 1.0 + 2.0 ** -8: 0x3F80, 1.0 + 3 * 2.0 ** -8: 0x3F82, 1.0 + 2.0 ** -8 + 2.0 ** -40: 0x3F81,
+        -2.5: 0xC020, 2.0 ** -133: 0x0001, 2.0 ** -134: 0x0000, 3 * 2.0 ** -134: 0x0002,
+        255.0 * 2.0 ** 120: 0x7F7F, 511.0 * 2.0 ** 119: 0x7F80, -1e39: 0xFF80, 0.0: 0x0000,
+    }
+    for val, bits in cases.items():
+        got = int(O.to_bf16(np.array([val]), _lib=lib)[0])
+        assert got == bits, (val, hex(got), hex(bits))
+
+
 ALL_CHECKS = [
     check_store_literal, check_store_roundtrip, check_store_rejects_out_of_range,
     check_one_token_returns_v, check_two_token_closed_form, check_explicit_scale, check_equal_keys_mean,
     check_brute_force, check_torch_sdpa, check_paging_contiguous, check_relabel, check_gqa_repeat,
     check_chunk_split, check_prefill_row_is_decode, check_prefix_sharing, check_nan_never_read,
     check_invalid_inputs, check_threads_agree,
+    check_rope_worked_example, check_rope_position_zero, check_rope_complex_product, check_rope_relative_position,
+    check_rope_strided_rows, check_to_bf16,
 ]

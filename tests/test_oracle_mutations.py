@@ -4,7 +4,9 @@ Each mutation is a one-line edit of oracle/oracle.c compiled into a temporary
 library (CPU only); the pins of tests/oracle_pins.py run against it and at
 least one must fail.  This shows the pins constrain every step of the oracle:
 the store's slot decoding, the gather, the head map, the scale, the causal
-position, the softmax normalisation and the value gather.
+position, the softmax normalisation, the value gather, the rotary embedding's
+direction, pairing, frequencies, positions and row addressing, and the bf16
+rounding.
 """
 
 import os
@@ -34,6 +36,16 @@ MUTATIONS = {
     "store_offset": ("const int64_t offset = s % block_size;", "const int64_t offset = s % block_size / 2;"),
     "store_skips_last_token": ("for (int32_t t = 0; t < num_tokens; ++t) {",
                                "for (int32_t t = 0; t + 1 < num_tokens; ++t) {"),
+    "rope_sin_sign": ("o[i] = x1 * c - x2 * s;", "o[i] = x1 * c + x2 * s;"),
+    "rope_adjacent_pairs": ("const double x2 = bf16_to_double(row[i + half]);",
+                            "const double x2 = bf16_to_double(row[half - 1 - i]);"),
+    "rope_frequency_exponent": ("pow(base, -2.0 * (double)i / (double)head_dim)",
+                                "pow(base, -(double)i / (double)head_dim)"),
+    "rope_position_shift": ("const double p = (double)positions[t];", "const double p = (double)positions[t] + 1.0;"),
+    "rope_head_stride": ("const uint16_t *row = x + t * token_stride + (int64_t)h * head_dim;",
+                         "const uint16_t *row = x + t * token_stride + (int64_t)h * half;"),
+    "bf16_round_down": ("ldexp(nearbyint(ldexp(a, -q)), q)", "ldexp(floor(ldexp(a, -q)), q)"),
+    "bf16_ties_away": ("ldexp(nearbyint(ldexp(a, -q)), q)", "ldexp(round(ldexp(a, -q)), q)"),
     "query_row_index": ("const uint16_t *qrow = job->q + (r * job->num_q_heads + hq) * (int64_t)D;",
                         "const uint16_t *qrow = job->q + (r * job->num_q_heads + hq % 2) * (int64_t)D;"),
 }
