@@ -635,7 +635,49 @@ def secondary(args, dev, stream, ops, W, timed):
         res[name] = r
         del st, ws, out, s
         torch.cuda.empty_cache()
+    res["qwen3_decode_rope"] = rope_decode(steps, dev, ops, W, timed)
     return res
+
+
+ROPE_BASE = 1.0e6  # Qwen3's rotary base
+
+
+def rope_decode(steps, dev, ops, W, timed):
+    """The headline decode step with RoPE: npv_rope_store_kvcache (rotate q in place,
+    rotate k, store k and v) then npv_paged_decode_attention, two launches per step."""
+    import torch
+
+    hbm_peak, _ = measured_peaks()
+    wl = W.workload(W.HEADLINE)
+    st = W.DeviceState(wl, dev)
+    s = st.steps[0]
+    _, pos = wl.token_positions(0)
+    positions = torch.from_numpy(pos.astype(np.int32)).to(dev)
+    q = s["q"].clone()
+    ws = ops.alloc_workspace(ops.decode_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.D), dev)
+    out = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device=dev)
+
+    def step(i):
+        ops.rope_store_kvcache(q, s["key"], s["value"], positions, st.k_cache, st.v_cache, s["slot_mapping"],
+                               ROPE_BASE)
+        ops.paged_decode_attention(q, st.k_cache, st.v_cache, s["block_tables"], s["context_lens"], out=out,
+                                   workspace=ws)
+
+    for i in range(3):
+        step(i)
+    ops.check_device_errors()
+    ms = timed(step, steps) / steps
+    ops.check_device_errors()
+    store_b, attn_b = step_bytes(wl, 0)
+    q_rt = 2 * wl.B * wl.Hq * wl.D * 2  # q read and rewritten by the rotation
+    gbs = (store_b + attn_b + q_rt) / (ms * 1e-3) / 1e9
+    r = {"metric": metric_for(wl), "ms_per_step": ms, "gb_s": gbs, "frac_of_hbm": gbs / hbm_peak,
+         "tokens_per_s": wl.B / (ms * 1e-3), "rope_base": ROPE_BASE,
+         "config": dict(workload_config(wl), workload="qwen3_decode with RoPE on q and k before the store"),
+         "bytes": "headline step bytes + the q rows read and rewritten by the rotation"}
+    del st, ws, out, s, q
+    torch.cuda.empty_cache()
+    return r
 
 
 def step_fn_kind(args, mixed):

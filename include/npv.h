@@ -116,6 +116,45 @@ NPV_API npv_status npv_store_kvcache(const void *key, const void *value, int64_t
                              npv_stream_t stream);
 
 /*
+ * Rotary position embedding of the new tokens' q and k, then the store of the
+ * rotated k and of v into their cache slots, in one launch ("Nano-vLLM
+ * Architecture and Performance", project structure: RoPE in
+ * layers/rotary_embedding.py, applied to q and k before the attention layer
+ * stores k and v; the store as for npv_store_kvcache).  The pages name RoPE
+ * without its formula; this is the rotary embedding of Su et al. ("RoFormer",
+ * section 3.4) in the rotate-half pairing that Qwen3 uses: for a row x of
+ * head_dim D at position p and i < D/2, the pair (x[i], x[i + D/2]) is turned
+ * by the angle p * theta_i, theta_i = rope_base^(-2i/D):
+ *     x[i]       <- x[i] cos - x[i + D/2] sin
+ *     x[i + D/2] <- x[i + D/2] cos + x[i] sin
+ * The angle, cos and sin are taken in double precision, the rotation in fp32,
+ * and each result is rounded to bf16 (nearest, ties to even) once.
+ *
+ *   q             [num_tokens, num_q_heads, head_dim] bf16, rows q_token_stride
+ *                 ELEMENTS apart (0: num_q_heads * head_dim); rotated IN PLACE.
+ *                 May be null when num_q_heads == 0 (k and v only).
+ *   key, value    [num_tokens, num_kv_heads, head_dim] bf16, strides as for
+ *                 npv_store_kvcache; read only (the rotated k goes to the cache).
+ *   positions     [num_tokens] int32 (device): token t's position (any int32;
+ *                 for a decode row, L_b - 1; for row i of an n_b-row chunk,
+ *                 L_b - n_b + i).
+ *   k_cache, v_cache, slot_mapping, num_blocks, block_size: as for
+ *                 npv_store_kvcache (a negative slot stores nothing, but the
+ *                 token's q rows are still rotated; a slot past the cache sets
+ *                 NPV_DEVERR_SLOT and stores nothing).
+ *   head_dim      a multiple of 16, at most 256 (else NPV_ERR_UNSUPPORTED).
+ *   rope_base     base of the frequencies (> 0 and finite; Qwen3 uses 1e6).
+ * All pointers 16-byte aligned, all strides * 2 bytes multiples of 16.
+ * num_tokens == 0 is a no-op.
+ */
+NPV_API npv_status npv_rope_store_kvcache(void *q, int64_t q_token_stride, int32_t num_q_heads, const void *key,
+                                          const void *value, int64_t key_token_stride, int64_t value_token_stride,
+                                          const int32_t *positions, void *k_cache, void *v_cache,
+                                          const int32_t *slot_mapping, int32_t num_tokens, int32_t num_blocks,
+                                          int32_t block_size, int32_t num_kv_heads, int32_t head_dim,
+                                          double rope_base, npv_stream_t stream);
+
+/*
  * Bytes of device workspace npv_paged_decode_attention needs on the current
  * device for this head configuration.  The size does not depend on context
  * lengths.  Returns 0 for arguments the call would reject.

@@ -14,6 +14,7 @@
 #include "npv.h"
 #include "npv_device.cuh"
 #include "store_kvcache.cuh"
+#include "rope_store.cuh"
 #include "decode_attention.cuh"
 #include "prefill_attention.cuh"
 
@@ -370,6 +371,52 @@ npv_status npv_store_kvcache(const void *key, const void *value, int64_t key_tok
     cudaError_t e = launch_pdl(npv::store::store_kvcache_kernel, dim3((unsigned)blocks),
                                dim3(npv::store::kThreads), 0, (cudaStream_t)stream, p);
     return cuda_status(e);
+}
+
+npv_status npv_rope_store_kvcache(void *q, int64_t q_token_stride, int32_t num_q_heads, const void *key,
+                                  const void *value, int64_t key_token_stride, int64_t value_token_stride,
+                                  const int32_t *positions, void *k_cache, void *v_cache,
+                                  const int32_t *slot_mapping, int32_t num_tokens, int32_t num_blocks,
+                                  int32_t block_size, int32_t num_kv_heads, int32_t head_dim, double rope_base,
+                                  npv_stream_t stream) {
+    if (num_tokens < 0 || num_q_heads < 0 || !cache_shape_ok(num_blocks, block_size, num_kv_heads, head_dim))
+        return NPV_ERR_INVALID_ARG;
+    if (!(rope_base > 0.0) || !std::isfinite(rope_base)) return NPV_ERR_INVALID_ARG;
+    if (head_dim % 16 != 0 || head_dim > npv::rope::kMaxHeadDim) return NPV_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return NPV_OK;
+    if (!key || !value || !k_cache || !v_cache || !slot_mapping || !positions) return NPV_ERR_INVALID_ARG;
+    if (num_q_heads > 0 && !q) return NPV_ERR_INVALID_ARG;
+    const int64_t kvrow = (int64_t)num_kv_heads * head_dim;
+    const int64_t qrow = (int64_t)num_q_heads * head_dim;
+    if (key_token_stride == 0) key_token_stride = kvrow;
+    if (value_token_stride == 0) value_token_stride = kvrow;
+    if (q_token_stride == 0) q_token_stride = qrow;
+    if (key_token_stride < kvrow || value_token_stride < kvrow || q_token_stride < qrow) return NPV_ERR_INVALID_ARG;
+    if ((key_token_stride * 2) % 16 != 0 || (value_token_stride * 2) % 16 != 0 || (q_token_stride * 2) % 16 != 0)
+        return NPV_ERR_INVALID_ARG;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (num_q_heads > 0 && !aligned16(q)))
+        return NPV_ERR_INVALID_ARG;
+    npv::rope::Params p = {};
+    p.q = num_q_heads > 0 ? static_cast<uint16_t *>(q) : nullptr;
+    p.q_stride = q_token_stride;
+    p.key = static_cast<const uint16_t *>(key);
+    p.value = static_cast<const uint16_t *>(value);
+    p.key_stride = key_token_stride;
+    p.value_stride = value_token_stride;
+    p.positions = positions;
+    p.slot_mapping = slot_mapping;
+    p.k_cache = static_cast<uint16_t *>(k_cache);
+    p.v_cache = static_cast<uint16_t *>(v_cache);
+    p.num_tokens = num_tokens;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.head_dim = head_dim;
+    p.num_slots = (int64_t)num_blocks * block_size;
+    p.base = rope_base;
+    const unsigned blocks = (unsigned)((num_tokens + npv::rope::kTokens - 1) / npv::rope::kTokens);
+    return cuda_status(launch_pdl(npv::rope::rope_store_kernel, dim3(blocks), dim3(npv::rope::kThreads), 0,
+                                  (cudaStream_t)stream, p));
 }
 
 size_t npv_paged_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,

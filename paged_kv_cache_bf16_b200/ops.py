@@ -59,6 +59,9 @@ def lib() -> C.CDLL:
     l.npv_version.restype = C.c_int
     l.npv_store_kvcache.argtypes = [p, p, i64, i64, p, p, p, i32, i32, i32, i32, i32, p]
     l.npv_store_kvcache.restype = C.c_int
+    l.npv_rope_store_kvcache.argtypes = [p, i64, i32, p, p, i64, i64, p, p, p, p, i32, i32, i32, i32, i32,
+                                         C.c_double, p]
+    l.npv_rope_store_kvcache.restype = C.c_int
     l.npv_paged_decode_workspace_size.argtypes = [i32, i32, i32, i32]
     l.npv_paged_decode_workspace_size.restype = sz
     l.npv_paged_decode_attention.argtypes = [p, p, i64, p, p, p, i32, p, i32, i32, i32, i32, i32, i32, C.c_float,
@@ -132,6 +135,29 @@ def store_kvcache(key: torch.Tensor, value: torch.Tensor, k_cache: torch.Tensor,
     _check(lib().npv_store_kvcache(_ptr(key), _ptr(value), key.stride(0) if T else 0, value.stride(0) if T else 0,
                                    _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping), T, NB, BS, Hkv, D,
                                    _stream(stream)), "npv_store_kvcache")
+
+
+def rope_store_kvcache(q: Optional[torch.Tensor], key: torch.Tensor, value: torch.Tensor, positions: torch.Tensor,
+                       k_cache: torch.Tensor, v_cache: torch.Tensor, slot_mapping: torch.Tensor, rope_base: float,
+                       stream=None) -> None:
+    """RoPE on q (in place, [T, Hq, D]; None for none) and key [T, Hkv, D] at positions [T] int32,
+    then the store of the rotated key and of value [T, Hkv, D] at slot_mapping [T] int32."""
+    _on_one_gpu("rope_store_kvcache",
+                bf16=[("q", q), ("key", key), ("value", value), ("k_cache", k_cache), ("v_cache", v_cache)],
+                other=[("positions", positions), ("slot_mapping", slot_mapping)])
+    NB, BS, Hkv, D = _cache_shape(k_cache)
+    T = slot_mapping.shape[0]
+    assert slot_mapping.dtype == torch.int32 and positions.dtype == torch.int32 and positions.shape == (T,)
+    assert key.shape[0] == T and value.shape[0] == T
+    assert key.stride(-1) == 1 and key.stride(-2) == D and value.stride(-1) == 1 and value.stride(-2) == D
+    Hq = 0 if q is None else q.shape[1]
+    if q is not None:
+        assert q.shape[0] == T and q.shape[2] == D and q.stride(-1) == 1 and q.stride(-2) == D
+    _check(lib().npv_rope_store_kvcache(_ptr(q) if q is not None else None, q.stride(0) if (q is not None and T) else 0,
+                                        Hq, _ptr(key), _ptr(value), key.stride(0) if T else 0,
+                                        value.stride(0) if T else 0, _ptr(positions), _ptr(k_cache), _ptr(v_cache),
+                                        _ptr(slot_mapping), T, NB, BS, Hkv, D, float(rope_base), _stream(stream)),
+           "npv_rope_store_kvcache")
 
 
 def decode_workspace_size(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int) -> int:
