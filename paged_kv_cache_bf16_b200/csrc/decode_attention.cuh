@@ -703,10 +703,17 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 1) decode_split_
 // invalid lengths) for sequences the split kernel had no chunks for.  The grid
 // has the split kernel's size.  Everything that does not read the split
 // kernel's output runs before griddepcontrol.wait, overlapping the split
-// kernel's tail; every CTA waits before it exits.
-__global__ void __launch_bounds__(256) decode_merge_kernel(const Params p, int head_dim) {
+// kernel's tail; every CTA waits before it exits.  Each thread's (row, 4
+// columns) item is two rounds of dependent loads (the partial maxima, then
+// the weighted sums), so the CTA is wide to keep many items' loads in flight:
+// a unit holds HC * g * n * D / 4 items (512 for 8 KV heads of 2 decode rows at
+// D = 128, 2,048 for 8 verification rows).  512 threads still fit on an SM
+// beside a split-kernel CTA, so the merge's schedule runs during the split
+// kernel's tail; 1,024 do not, and pay off only for multi-row units.
+template <int kThreadsM>
+__global__ void __launch_bounds__(kThreadsM) decode_merge_kernel(const Params p, int head_dim) {
     __shared__ long long sched[4];
-    __shared__ long long scratch[16];
+    __shared__ long long scratch[kThreadsM / 32 + 1];
     const int D = head_dim;
     const long long c = blockIdx.x;
     const long long G = gridDim.x;

@@ -80,6 +80,7 @@ struct DecodeConfig {
     int max_rows = 0;        // most query rows of a sequence the kernel serves
     int rows_per_head = 0;   // partial-slot rows per KV head: g * max_rows
     bool sole_path = false;  // mixed batch with no prefill kernel launched
+    bool wide_merge = false; // merge CTAs of 1,024 threads (units of many query rows)
     int stages = 0;
     int grid = 0;
     size_t smem = 0;
@@ -212,7 +213,11 @@ npv_status run_decode(void *out, const void *q, int64_t q_row_stride, const int3
     }
     cudaError_t e = dispatch_decode_split(head_dim, p, cfg, stream);
     if (e != cudaSuccess) return NPV_ERR_CUDA;
-    e = launch_pdl(npv::decode::decode_merge_kernel, dim3(cfg.grid), dim3(256), 0, stream, p, (int)head_dim);
+    if (cfg.wide_merge)
+        e = launch_pdl(npv::decode::decode_merge_kernel<1024>, dim3(cfg.grid), dim3(1024), 0, stream, p,
+                       (int)head_dim);
+    else
+        e = launch_pdl(npv::decode::decode_merge_kernel<512>, dim3(cfg.grid), dim3(512), 0, stream, p, (int)head_dim);
     return cuda_status(e);
 }
 
@@ -536,6 +541,9 @@ npv_status npv_paged_prefill_attention(void *out, const void *q, const int32_t *
     // sequence is left for the tensor-memory kernel: its plan and launch are
     // skipped, and the decode kernel reports a sequence that breaks the bound.
     cfg.decode.sole_path = max_seqlen_q <= cfg.decode.max_rows;
+    // a call of multi-row sequences only (speculative-decode verification) has
+    // merges of g * n_b >= 8 rows per KV head: the wide merge CTA
+    cfg.decode.wide_merge = cfg.decode.sole_path && (int64_t)max_seqlen_q * G >= 8;
     if (!cfg.decode.sole_path) {
         // tensor maps, 128-byte swizzle: the caches [NB * BS, Hkv, D] in boxes of
         // {64 elements, 1 head, box_tokens slots}; q [total_q, Hq, D] in boxes of

@@ -7,47 +7,49 @@
 // are already stored at positions L_b - n_b .. L_b - 1, row i attends to keys
 // 0 .. L_b - n_b + i of the sequence's paged K/V, query head h reading KV head
 // h / g, scale 1/sqrt(D) by default.  This kernel takes the sequences with
-// n_b > 16 / g; shorter ones (decode rows, speculative-decode verification)
-// go to the split-KV decode kernel in the same call.
+// more query rows than the split-KV decode kernel's tile holds (n_b > 16 / g,
+// or 8 / g when the call's bound on n_b allows the lighter decode variant);
+// shorter ones (decode rows, speculative-decode verification) go to the
+// decode kernel in the same call.
 //
 // How (B200 design):
-//   * Work item = (sequence, KV head, tile of 128 MMA rows).  The 128 rows pack
-//     128/g positions x the g query heads of one GQA group, so every K/V tile
-//     loaded from HBM feeds all g heads (row r = position * g + head).
-//   * A one-CTA plan kernel lists the (sequence, row-tile) pairs: sequences
-//     counting-sorted by KV length, longest first, each sequence's tiles
+//   * Q tiles: 128 MMA rows pack 128/g positions x the g query heads of one
+//     GQA group, so every K/V tile loaded feeds all g heads (row r = position *
+//     g + head).  A work item is (sequence, KV head, pair of consecutive Q
+//     tiles A and B): both Q tiles share every K/V tile the CTA loads, which
+//     halves the K/V traffic from L2 against one Q tile per item.
+//   * A one-CTA plan kernel lists the (sequence, pair) entries: sequences
+//     counting-sorted by KV length, longest first, each sequence's pairs
 //     contiguous (so the items that read the same K/V run at the same time and
 //     share it through L2).  The persistent main kernel (one CTA per SM) takes
-//     items (pair, KV head) from that list in snake order.
-//   * Measured on B200: one tcgen05.mma M128 x N128 x K16 runs 64 cycles, but
-//     the issuing thread spends ~48 cycles per MMA instruction, ~50 per commit
-//     and ~58 per mbarrier wait.  One Q tile of 128 rows gives the issuer 16
-//     MMAs + 3 commits + 4 waits per 128-key tile, about the 1,024 cycles the
-//     tensor pipe needs for it, so the issuer's loop has no slack to spare: it
-//     issues S_{t+2} right after P_t V_t, and waits have a one-instruction fast
-//     path.
-//   * Split KV inside the CTA: softmax warpgroup j (warps 4-7, 8-11) takes the
-//     KV tiles T with T % 2 == j, with its own S buffer, running (max, sum) and
-//     O accumulator; the two partial results are merged in the epilogue.  The
-//     warpgroups never wait for each other inside the KV loop and their
-//     exponential phases interleave on the special-function units.
+//     items (entry, KV head) from that list in snake order.
 //   * Warp roles: warp 0 owns tensor memory and issues tcgen05.mma from one
 //     thread; warp 1 issues the TMA loads of the K tiles (128 keys) through a
-//     3-stage ring, warp 2 those of the V tiles through a 3-stage ring (block ids
-//     from the block table a 32-entry window at a time, one TMA box per block
-//     piece); warp 3 loads each item's Q tile with one TMA box per 64 columns.
-//     The first warpgroup gives registers to the softmax warpgroups (setmaxnreg)
-//     so that a softmax thread holds a whole 128-key row of S.
+//     2-stage ring, warp 2 those of the V tiles through a 3-stage ring (block
+//     ids from the block table a 32-entry window at a time, one TMA box per
+//     block piece); warp 3 loads each item's two Q tiles.  Softmax warpgroup j
+//     (warps 4-7 for A, 8-11 for B) owns Q tile j: its S buffer, running (max,
+//     sum) and O accumulator, and writes its tile's output rows.  The first
+//     warpgroup gives registers to the softmax warpgroups (setmaxnreg) so that
+//     a softmax thread holds a whole 128-key row of S.
+//   * Per KV tile t the MMA thread issues O_A += P_A(t) V_t, S_A(t+1), O_B +=
+//     P_B(t) V_t, S_B(t+1): while softmax warpgroup A works on its tile the
+//     tensor pipe runs B's products, and the other way round.
+//   * Measured on B200: one tcgen05.mma M128 x N128 x K16 runs 64 cycles, and
+//     the issuing thread spends ~48 cycles per MMA instruction, ~50 per commit
+//     and ~58 per mbarrier wait.  Timing experiments put the kernel's limit in
+//     the barrier round trips of each step (S ready -> softmax -> P ready ->
+//     the next products), not in the loads, the tensor pipe or `ex2`.
 //   * Operands: S = Q K^T reads Q and K from shared memory (K-major, 128-byte
 //     swizzle); P V reads P from tensor memory, where the softmax writes it as
 //     bf16 pairs over the first 64 columns of its own S buffer, and V from
-//     shared memory (MN-major).  Tensor memory (512 columns): S_0, S_1 (128
-//     fp32 columns each), O_0, O_1 (D columns each).
+//     shared memory (MN-major).  Tensor memory (512 columns): S_A, S_B (128
+//     fp32 columns each), O_A, O_B (D columns each, at 256 and 384).
 //   * The softmax keeps a per-row running max in the log2 domain and rescales
 //     its O accumulator only when the max grows by more than 2^8 (otherwise the
 //     stale max is kept; the final division by the row sum corrects it exactly
 //     in real arithmetic).  V rows past the context of the last tile are zeroed
-//     before the P.V product so unwritten cache slots never meet it; rows of the
+//     before the P.V product so unwritten cache slots never meet it; rows of a
 //     tile past its positions attend like its first row and are not stored.
 #pragma once
 
@@ -88,8 +90,8 @@ struct Params {
     int32_t box_tokens;  // tokens per K/V TMA box: 128 when block_size % 128 == 0, else 16
     const uint16_t *q;   // [total_q, Hq, D]
     float scale_log2;
-    int32_t *plan_count;  // [1]: number of (sequence, row-tile) pairs
-    int2 *plan_pairs;     // [max_pairs]: (sequence, row tile), longest first
+    int32_t *plan_count;  // [1]: number of (sequence, pair of Q tiles) entries
+    int2 *plan_pairs;     // [max_pairs]: (sequence, index of the pair of Q tiles), longest first
     int32_t max_pairs;
     int32_t decode_rows_max;  // sequences with at most this many query rows run on the decode kernel
 };
@@ -150,7 +152,7 @@ __device__ __forceinline__ long long item_index(long long r) {
 }
 
 // A sequence runs on this kernel when it has more query rows than the decode
-// kernel's warp-level tile takes (n_b > decode_rows_max = 16 / g).
+// kernel's warp-level tile takes (n_b > decode_rows_max: 16 / g or 8 / g).
 __device__ __forceinline__ bool prefill_seq(const Params &p, int32_t b, int32_t *n_out, bool *bad) {
     const int32_t cb = __ldg(p.cu_seqlens_q + b), ce = __ldg(p.cu_seqlens_q + b + 1);
     *bad = false;
@@ -206,7 +208,7 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const Params p, int 
     (void)base;
     __syncthreads();
     // Sequences are ordered by their KV length, longest first (counting sort on
-    // 128-key tiles); each sequence's row tiles stay contiguous, last tile first,
+    // 128-key tiles); each sequence's pairs of Q tiles stay contiguous, last first,
     // so the CTAs reading the same K/V run together and share it through L2.
     for (int b = lo; b < hi; ++b) {
         int32_t n;
@@ -249,7 +251,7 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const Params p, int 
             if (pos + k < p.max_pairs) p.plan_pairs[pos + k] = make_int2(b, nqt - 1 - k);
     }
     if (tid == 0) {
-        // cu_seqlens_q must run from 0 to total_q; a list of row tiles longer than
+        // cu_seqlens_q must run from 0 to total_q; a list of entries longer than
         // the plan can hold means ranges overlap (some entry decreased).  Either
         // way the call's rows are not a partition of q: report it.  The plan is
         // clamped, so no access leaves the workspace.
