@@ -35,11 +35,13 @@
 //   * Per KV tile t the MMA thread issues O_A += P_A(t) V_t, S_A(t+1), O_B +=
 //     P_B(t) V_t, S_B(t+1): while softmax warpgroup A works on its tile the
 //     tensor pipe runs B's products, and the other way round.
-//   * Measured on B200: one tcgen05.mma M128 x N128 x K16 runs 64 cycles, and
-//     the issuing thread spends ~48 cycles per MMA instruction, ~50 per commit
-//     and ~58 per mbarrier wait.  Timing experiments put the kernel's limit in
-//     the barrier round trips of each step (S ready -> softmax -> P ready ->
-//     the next products), not in the loads, the tensor pipe or `ex2`.
+//   * Measured on B200: one tcgen05.mma M128 x N128 x K16 runs 64 cycles, but
+//     the issuing thread, on a sub-partition shared with two busy softmax
+//     warps, spends ~120 cycles per MMA instruction (traced in this kernel):
+//     the single issuer paces the kernel, not the loads, the barrier hops
+//     (~110 cycles), the tensor pipe or `ex2`.  One issuer per Q tile was
+//     slower: the two tiles' products interleave in the tensor pipe and the
+//     softmax warpgroups stop alternating with them.
 //   * Operands: S = Q K^T reads Q and K from shared memory (K-major, 128-byte
 //     swizzle); P V reads P from tensor memory, where the softmax writes it as
 //     bf16 pairs over the first 64 columns of its own S buffer, and V from
