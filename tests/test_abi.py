@@ -52,6 +52,31 @@ def test_host_validation_before_any_cuda_call(lib):
                                           0, None) == 1
 
 
+def test_rope_store_host_validation(lib):
+    f = lib.npv_rope_store_kvcache
+    # (q, q_stride, Hq, key, value, k_stride, v_stride, positions, k_cache, v_cache, slots, T, NB, BS, Hkv, D,
+    #  base, stream)
+    ok = dict(T=0, D=64, base=1.0e6)
+
+    def call(T=0, D=64, base=1.0e6, hq=2):
+        return f(None, 0, hq, None, None, 0, 0, None, None, None, None, T, 8, 16, 2, D, base, None)
+
+    assert call(**ok) == 0                   # no tokens: a no-op
+    assert call(T=-1) == 1                   # negative count
+    assert call(T=4) == 1                    # null pointers
+    assert call(base=0.0) == 1               # the base must be positive and finite
+    assert call(base=float("nan")) == 1
+    assert call(base=float("inf")) == 1
+    assert call(D=40) == 2                   # head_dim not a multiple of 16
+    assert call(D=512) == 2                  # above 256
+    assert call(hq=-1) == 1
+
+
+def test_prefill_rejects_a_negative_row_bound(lib):
+    assert lib.npv_paged_prefill_attention(None, None, None, -1, 8, None, None, None, 4, None, 2, 4, 2, 64, 8, 16,
+                                           0.0, None, 0, None) == 1
+
+
 def test_python_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     code = ("import paged_kv_cache_bf16_b200.ops as o; o.LIB_PATH = %r\n"
             "try:\n    o.lib()\nexcept RuntimeError as e:\n    print('raised', e)\n") % str(tmp_path / "nope.so")
