@@ -2,9 +2,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl npv|reference] [--workload NAME]
 
-One step = one decode step of the workload: npv_store_kvcache of this step's
-new K/V rows, then npv_paged_decode_attention (split-KV kernel + merge kernel)
-over every sequence.  The default workload is the Qwen3-0.6B-shaped decode
+One step = one decode step of the workload: npv_store_kvcache_and_decode_attention
+(the store of this step's new K/V rows inside the split-KV kernel, then the merge
+kernel) over every sequence; --separate-store runs npv_store_kvcache then
+npv_paged_decode_attention instead.  The default workload is the Qwen3-0.6B-shaped decode
 batch (256 sequences, 16 Q / 8 KV heads, head_dim 128, 256-token blocks,
 contexts U[100, 2048] growing by one token per step, cycling through its 64
 steps).  Inputs are synthetic and seeded; the KV read per step (about 1.16 GB)
@@ -13,6 +14,11 @@ is far larger than the 126 MB L2, so no explicit flush is needed.
 `value` is algorithmic HBM bytes per step / device time per step (GB/s), summed
 over ranks for N > 1 (each rank runs its own replica; no collective on the data
 path) and divided by the slowest rank's time.  Prints one JSON line on rank 0.
+
+At N = 1 the default run then times every other named workload (GQA 4:1 with
+shared prefixes, long-context decode, the chunked-prefill mix, speculative-decode
+verification) and the decode step with RoPE, one short loop each, in the line's
+`secondary` block.
 
 --impl reference times the fp64 CPU oracle (the only reference this method
 has) on a bounded sample of the same workload, on rank 0 only.
